@@ -1,0 +1,86 @@
+"""ctypes loader for libgnorm.so (the C ABI declared in include/gnorm.h).
+
+The shared library is built in-tree (``python -m gated_norm_b200.build``).  There is no
+fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgnorm.so")
+
+GNORM_OK = 0
+GNORM_ERR_NULL = -1
+GNORM_ERR_SHAPE = -2
+GNORM_ERR_ALIGN = -3
+GNORM_ERR_ALIAS = -4
+GNORM_ERR_UNSUPPORTED = -5
+GNORM_ERR_WORKSPACE = -6
+GNORM_ERR_CUDA = -7
+GNORM_ERR_ARG = -8
+GNORM_N_MAX = 16384
+GNORM_WORKSPACE_ALIGN = 256
+
+
+class GnormPlan(ctypes.Structure):
+    """Mirror of ``gnorm_plan`` in include/gnorm.h."""
+
+    _fields_ = [
+        ("kind", ctypes.c_int),
+        ("threads_per_row", ctypes.c_int),
+        ("chunks_per_thread", ctypes.c_int),
+        ("consumer_threads", ctypes.c_int),
+        ("rows_per_stage", ctypes.c_int),
+        ("stages", ctypes.c_int),
+        ("ctas_per_sm", ctypes.c_int),
+        ("grid", ctypes.c_int),
+        ("num_blocks", ctypes.c_int64),
+        ("smem_bytes", ctypes.c_int),
+        ("dynamic_schedule", ctypes.c_int),
+        ("fused_reduce", ctypes.c_int),
+        ("partials", ctypes.c_int),
+        ("reserved", ctypes.c_int),
+    ]
+
+    def as_dict(self) -> dict:
+        return {name: getattr(self, name) for name, _ in self._fields_ if name != "reserved"}
+
+
+_vp = ctypes.c_void_p
+_i64 = ctypes.c_int64
+_int = ctypes.c_int
+_f32 = ctypes.c_float
+_sz = ctypes.c_size_t
+
+# name -> (restype, argtypes); every symbol include/gnorm.h declares.
+SIGNATURES = {
+    "gnorm_fwd": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _i64, _i64, _vp]),
+    "gnorm_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _vp, _sz,
+                         _vp]),
+    "gnorm_ckpt_step": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
+                               _i64, _vp, _sz, _vp]),
+    "gnorm_bwd_workspace_bytes": (_sz, [_i64, _i64, _int]),
+    "gnorm_bwd_workspace_bytes_for": (_sz, [_i64, _i64, _int, _int]),
+    "gnorm_status_string": (ctypes.c_char_p, [_int]),
+    "gnorm_plan_query": (_int, [_int, _i64, _i64, _int, _int, _int, ctypes.POINTER(GnormPlan)]),
+    "gnorm_device_error": (_int, [_int]),
+    "gnorm_set_tuning": (None, [_int, _int, _int, _int]),
+    "gnorm_build_info": (ctypes.c_char_p, []),
+}
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(
+            f"{path} is missing: build it with `python -m gated_norm_b200.build` "
+            "(the CUDA path has no CPU fallback)")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+lib = load()

@@ -1,0 +1,329 @@
+// bwd_kernel.cuh -- backward of the SiLU-gated RMSNorm on sm_100a, and the dw reduction.
+//
+// Per row, with the forward's FP32 rstd r:  xhat = x r,  s = g sigmoid(g),  u = dy w s,
+// c = mean(u xhat),  dx = r (u - xhat c),  dg = dy xhat w sigmoid(g) (1 + g (1 - sigmoid(g))),
+// and dw = sum over rows of dy xhat s.  (flashinfer PR #8701, "perf(cake_rmsnorm_silu_gate_
+// train): L2-prefetching extra-long forward on SM107", section "How the tables were
+// measured": "bwdg" / "bwdg_f32" -- the backward with a BF16 / FP32 dw; the deterministic
+// package gives run-to-run bitwise results.  The fixed-order FP32 partial reduction follows
+// the pattern described in flashinfer PR #8878's commit message: per-CTA FP32 accumulators
+// reduced in a fixed order.)
+//
+// Design: the same persistent, warp-specialised TMA pipeline as the forward, with three
+// tensors (dy, x, g) per stage.  Pass 1 recomputes xhat and the gate from shared memory,
+// writes dg, accumulates the row dot product sum(u xhat) and this thread's dw columns in
+// FP32 registers, and keeps u in registers; after the row reduction pass 2 re-reads x and
+// writes dx.  At the end each CTA adds its row groups' dw accumulators in a fixed order into one
+// FP32 partial row [P, N] in the workspace.  A second launch (or, in the non-deterministic
+// mode for narrow rows, the last CTA to finish) sums the P partials in a fixed tree order
+// and writes dw once, rounded to BF16 or kept in FP32.
+#pragma once
+
+#include "args.h"
+#include "device_common.cuh"
+
+namespace gnorm {
+
+
+// Sums P rows of FP32 partials [P, N] into dw[N] in a fixed order: thread (bl, q) adds
+// rows bl, bl + BL, bl + 2 BL, ... of column quad q, then the BL lanes are combined by a
+// binary tree (BL = nthreads / 32, a power of two).  `scratch` holds nthreads float4.
+template <bool kNamedBarrier>
+__device__ __forceinline__ void reduce_partials(const float* __restrict__ partial, int P, int N,
+                                                void* dw, int dw_fp32, int col_tile0,
+                                                int col_tile_step, int tid, int nthreads,
+                                                float4* scratch) {
+  const int BL = nthreads >> 5;
+  const int bl = tid >> 5;
+  const int q = tid & 31;
+  const int n4 = N >> 2;
+  auto sync = [&]() {
+    if constexpr (kNamedBarrier)
+      named_barrier_sync(15, nthreads);
+    else
+      __syncthreads();
+  };
+  for (int t0 = col_tile0; t0 < n4; t0 += col_tile_step) {
+    const int j4 = t0 + q;
+    const bool valid = j4 < n4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (valid) {
+      const float4* p4 = reinterpret_cast<const float4*>(partial) + j4;
+      for (int b = bl; b < P; b += BL) {
+        const float4 v = __ldcg(p4 + static_cast<size_t>(b) * n4);
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+    }
+    scratch[tid] = acc;
+    sync();
+    for (int st = BL >> 1; st > 0; st >>= 1) {
+      if (bl < st) {
+        const float4 o = scratch[tid + st * 32];
+        float4 m = scratch[tid];
+        m.x += o.x;
+        m.y += o.y;
+        m.z += o.z;
+        m.w += o.w;
+        scratch[tid] = m;
+      }
+      sync();
+    }
+    if (bl == 0 && valid) {
+      const float4 m = scratch[q];
+      if (dw_fp32) {
+        reinterpret_cast<float4*>(dw)[j4] = m;
+      } else {
+        uint2 h;
+        h.x = pack_bf16x2(m.x, m.y);
+        h.y = pack_bf16x2(m.z, m.w);
+        reinterpret_cast<uint2*>(dw)[j4] = h;
+      }
+    }
+    sync();
+  }
+}
+
+// Second pass of the deterministic dw: one CTA per 128 columns.  Also clears the
+// dynamic-schedule counter of the workspace (the backward grid has finished by now).
+__global__ void __launch_bounds__(kReduceThreads)
+    dw_reduce_kernel(const float* __restrict__ partial, int P, int N, void* dw, int dw_fp32,
+                     unsigned long long* work_counter) {
+  __shared__ float4 scratch[kReduceThreads];
+  grid_dependency_wait();
+  allow_dependent_launch();
+  reduce_partials<false>(partial, P, N, dw, dw_fp32, blockIdx.x * 32, gridDim.x * 32,
+                         threadIdx.x, kReduceThreads, scratch);
+  if (work_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0ull;
+}
+
+template <int TPR, int CPT>
+__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
+    gated_rmsnorm_bwd_kernel(const BwdArgs a) {
+  constexpr int kNCT = consumer_threads_for(TPR);
+  constexpr int kGroups = kNCT / TPR;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  long long* blk_id = reinterpret_cast<long long*>(smem + 256);
+  int* last_flag = reinterpret_cast<int*>(smem + 384);
+  float* red_slots = reinterpret_cast<float*>(smem + kRedSlotOffset);
+  uint8_t* stage0 = smem + kHeaderBytes;
+
+  const int S = a.stages;
+  const int R = a.rows_per_stage;
+  const int N = a.N;
+  const uint32_t tensor_bytes = static_cast<uint32_t>(R) * N * 2u;
+  const uint32_t stage_bytes = (3u * tensor_bytes + 127u) & ~127u;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kNCT / 32);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  grid_dependency_wait();
+  allow_dependent_launch();
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0) {
+    // ---------------- producer ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t phase = 0;
+      long long next = blockIdx.x;
+      while (true) {
+        const long long blk =
+            a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
+        next += gridDim.x;
+        if (!mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty)) break;
+        if (blk >= a.num_blocks) {
+          blk_id[s] = -1;
+          mbar_arrive(&full[s]);
+          break;
+        }
+        blk_id[s] = blk;
+        const long long r0 = blk * R;
+        const long long left = a.M - r0;
+        const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
+        const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+        uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
+        mbar_arrive_expect_tx(&full[s], 3u * bytes);
+        bulk_copy_g2s(st, a.dy + r0 * N, bytes, &full[s]);
+        bulk_copy_g2s(st + tensor_bytes, a.x + r0 * N, bytes, &full[s]);
+        bulk_copy_g2s(st + 2u * tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+        if (++s == S) {
+          s = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int ctid = threadIdx.x - 32;
+  const int group = ctid / TPR;
+  const int lr = ctid - group * TPR;
+  const int n8 = N >> 3;
+
+  float wf[CPT][8];
+  float dwacc[CPT][8];
+  bool cval[CPT];
+#pragma unroll
+  for (int k = 0; k < CPT; ++k) {
+    const int c = k * TPR + lr;
+    cval[k] = c < n8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      wf[k][e] = 0.f;
+      dwacc[k][e] = 0.f;
+    }
+    if (cval[k]) bf16x8_to_f32(*reinterpret_cast<const uint4*>(a.w + c * 8), wf[k]);
+  }
+
+  int s = 0;
+  uint32_t phase = 0;
+  int slot = 0;
+  while (true) {
+    if (!mbar_wait(&full[s], phase, a.err, kErrWaitFull)) break;
+    const long long blk = blk_id[s];
+    if (blk < 0) break;
+    const long long r0 = blk * R;
+    const long long left = a.M - r0;
+    const int rows = static_cast<int>(left < R ? left : R);
+    const uint8_t* sdy = stage0 + static_cast<size_t>(s) * stage_bytes;
+    const uint8_t* sx = sdy + tensor_bytes;
+    const uint8_t* sg = sx + tensor_bytes;
+
+    for (int rb = 0; rb < rows; rb += kGroups) {
+      const int row = rb + group;
+      const bool valid = row < rows;
+      const int srow = valid ? row : 0;
+      const size_t roff = static_cast<size_t>(srow) * N * 2;
+      const long long grow = r0 + row;
+      const float r = valid ? __ldg(a.rstd + grow) : 0.f;
+
+      // pass 1: recompute xhat and the gate; dg; row dot product; dw accumulators
+      float u[CPT][8];
+      float dot = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        if (cval[k]) {
+          const int c = k * TPR + lr;
+          const size_t off = roff + static_cast<size_t>(c) * 16;
+          float dyf[8], xf[8], gf[8], dgf[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sdy + off), dyf);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sx + off), xf);
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sg + off), gf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float xhat = xf[e] * r;
+            const float sgm = sigmoid_f32(gf[e]);
+            const float silu = gf[e] * sgm;
+            const float t = dyf[e] * xhat;                   // dy xhat
+            const float ue = (dyf[e] * wf[k][e]) * silu;      // dy w s
+            u[k][e] = ue;
+            dot = fmaf(ue, xhat, dot);
+            dwacc[k][e] = valid ? fmaf(t, silu, dwacc[k][e]) : dwacc[k][e];
+            dgf[e] = ((t * wf[k][e]) * sgm) * ((1.0f + gf[e]) - silu);
+          }
+          if (valid)
+            *reinterpret_cast<uint4*>(a.dg + grow * N + c * 8) = f32x8_to_bf16(dgf);
+        }
+      }
+      dot = row_sum<TPR>(dot, red_slots, group, lr, slot);
+      slot ^= 1;
+      const float rc = r * (dot * a.inv_n);
+
+      // pass 2: dx = r u - (r c) xhat, with xhat recomputed from the staged x (this keeps
+      // u, w and the dw accumulators as the only per-element registers)
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        if (cval[k]) {
+          const int c = k * TPR + lr;
+          float xf[8], dxf[8];
+          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(c) * 16),
+                        xf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) dxf[e] = fmaf(-rc, xf[e] * r, r * u[k][e]);
+          if (valid)
+            *reinterpret_cast<uint4*>(a.dx + grow * N + c * 8) = f32x8_to_bf16(dxf);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == S) {
+      s = 0;
+      phase ^= 1u;
+    }
+  }
+
+  // ---------------- this CTA's dw partial: row groups added in a fixed order ----------------
+  named_barrier_sync(15, kNCT);  // every consumer is done with the stage buffers
+  float* prow = a.partial + static_cast<size_t>(blockIdx.x) * N;
+  if constexpr (kGroups == 1) {
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+      if (cval[k]) {
+        float4* p4 = reinterpret_cast<float4*>(prow + (k * TPR + lr) * 8);
+        p4[0] = make_float4(dwacc[k][0], dwacc[k][1], dwacc[k][2], dwacc[k][3]);
+        p4[1] = make_float4(dwacc[k][4], dwacc[k][5], dwacc[k][6], dwacc[k][7]);
+      }
+    }
+  } else {
+    float* red = reinterpret_cast<float*>(stage0);  // [kGroups, N]
+#pragma unroll
+    for (int k = 0; k < CPT; ++k) {
+      if (cval[k]) {
+        float4* r4 = reinterpret_cast<float4*>(red + group * N + (k * TPR + lr) * 8);
+        r4[0] = make_float4(dwacc[k][0], dwacc[k][1], dwacc[k][2], dwacc[k][3]);
+        r4[1] = make_float4(dwacc[k][4], dwacc[k][5], dwacc[k][6], dwacc[k][7]);
+      }
+    }
+    named_barrier_sync(15, kNCT);
+    const int n4 = N >> 2;
+    const float4* red4 = reinterpret_cast<const float4*>(red);
+    for (int j4 = ctid; j4 < n4; j4 += kNCT) {
+      float4 acc = red4[j4];
+#pragma unroll
+      for (int gi = 1; gi < kGroups; ++gi) {
+        const float4 v = red4[gi * n4 + j4];
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      reinterpret_cast<float4*>(prow)[j4] = acc;
+    }
+  }
+
+  if (!a.fused_reduce) return;
+
+  // ---------------- fused tail: the last CTA to finish sums all partials ----------------
+  __threadfence();
+  named_barrier_sync(15, kNCT);
+  if (ctid == 0) {
+    const unsigned done = atomicAdd(a.ticket, 1u);
+    *last_flag = (done == gridDim.x - 1) ? 1 : 0;
+  }
+  named_barrier_sync(15, kNCT);
+  if (*last_flag) {
+    __threadfence();
+    float4* scratch = reinterpret_cast<float4*>(stage0 + static_cast<size_t>(kGroups) * N * 4);
+    reduce_partials<true>(a.partial, gridDim.x, N, a.dw, a.dw_fp32, 0, 32, ctid, kNCT, scratch);
+    if (ctid == 0) {
+      *a.work_counter = 0ull;
+      *a.ticket = 0u;
+    }
+  }
+}
+
+}  // namespace gnorm

@@ -1,0 +1,166 @@
+// device_common.cuh -- sm_100a building blocks shared by the gated-norm kernels:
+// mbarrier pipeline waits with a time limit, 1-D TMA bulk copies (cp.async.bulk),
+// programmatic dependent launch, BF16 packing and the logistic function.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "layout.h"
+
+namespace gnorm {
+
+// Bits of the device error word (see gnorm_device_error in include/gnorm.h).
+constexpr unsigned kErrWaitFull = 1u;   // a consumer gave up waiting for copied rows
+constexpr unsigned kErrWaitEmpty = 2u;  // the producer gave up waiting for a free stage
+
+// A pipeline wait that has not completed after this long is abandoned.  A stage of a
+// few tens of KB arrives in microseconds, so two seconds only trips on a real fault.
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
+               : "memory");
+}
+
+// Makes barrier initialisation visible to the asynchronous (TMA) proxy.
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar_addr), "r"(parity)
+      : "memory");
+  return done != 0;
+}
+
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Waits until the barrier phase with the given parity has completed.  Gives up after
+// kWaitLimitNs (or 2^24 polling rounds, whichever comes first), sets `err_bit` in the
+// device error word and returns false; the caller then stops its loop and exits.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err_word,
+                                          unsigned err_bit) {
+  const uint32_t a = smem_u32(bar);
+  if (mbar_try_wait(a, parity)) return true;
+  const unsigned long long t0 = globaltimer_ns();
+  for (uint32_t round = 0; round < (1u << 24); ++round) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(a, parity)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+  }
+  atomicOr(err_word, err_bit);
+  return false;
+}
+
+// 1-D bulk copy global -> shared through the TMA unit; completion is counted in bytes on
+// `bar`.  Both addresses must be 16-byte aligned and `bytes` a multiple of 16.  No
+// multicast: the source is always this GPU's memory and only this CTA receives it.
+__device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_src,
+                                              uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Programmatic dependent launch: wait for the previous grid on the stream to complete
+// (and its memory to be visible) / allow the next grid to begin launching.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void allow_dependent_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// Eight BF16 values in a 16-byte word -> FP32 (exact: BF16 is the high half of FP32).
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 v, float f[8]) {
+  f[0] = __uint_as_float(v.x << 16);
+  f[1] = __uint_as_float(v.x & 0xffff0000u);
+  f[2] = __uint_as_float(v.y << 16);
+  f[3] = __uint_as_float(v.y & 0xffff0000u);
+  f[4] = __uint_as_float(v.z << 16);
+  f[5] = __uint_as_float(v.z & 0xffff0000u);
+  f[6] = __uint_as_float(v.w << 16);
+  f[7] = __uint_as_float(v.w & 0xffff0000u);
+}
+
+// Two FP32 -> two BF16 (round to nearest even), `lo` at the lower address.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float f[8]) {
+  uint4 v;
+  v.x = pack_bf16x2(f[0], f[1]);
+  v.y = pack_bf16x2(f[2], f[3]);
+  v.z = pack_bf16x2(f[4], f[5]);
+  v.w = pack_bf16x2(f[6], f[7]);
+  return v;
+}
+
+// Logistic function 1 / (1 + e^-t) with the fast exponential and the approximate
+// division intrinsics (one MUFU exp2 and one MUFU reciprocal).  Relative error is a few
+// FP32 ulp; for t < -88 the result is 0 (true value < 1e-38), for large t it is 1.
+__device__ __forceinline__ float sigmoid_f32(float t) {
+  return __fdividef(1.0f, 1.0f + __expf(-t));
+}
+
+// Sum over the `TPR` consecutive threads that share a row.  TPR <= 32: butterfly
+// shuffles inside the warp (every lane of the warp must call).  TPR > 32: butterfly per
+// warp, then the warps of the row exchange partials through shared-memory slots guarded
+// by a named barrier; `slot` alternates between two buffers from row to row so a fast
+// warp cannot overwrite slots a slow warp still reads.  The order of additions is fixed,
+// and every thread of the row ends with the bitwise same value.
+template <int TPR>
+__device__ __forceinline__ float row_sum(float v, float* red_slots, int group, int lane_in_row,
+                                         int slot) {
+#pragma unroll
+  for (int off = (TPR < 32 ? TPR : 32) / 2; off > 0; off >>= 1)
+    v += __shfl_xor_sync(0xffffffffu, v, off);
+  if constexpr (TPR > 32) {
+    constexpr int kWarps = TPR / 32;
+    const int wig = lane_in_row >> 5;  // warp index inside the row's thread group
+    float* slots = red_slots + (group * 2 + slot) * kWarps;
+    if ((lane_in_row & 31) == 0) slots[wig] = v;
+    named_barrier_sync(1 + group, TPR);
+    v = slots[0];
+#pragma unroll
+    for (int i = 1; i < kWarps; ++i) v += slots[i];
+  }
+  return v;
+}
+
+}  // namespace gnorm

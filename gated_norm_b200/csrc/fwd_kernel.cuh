@@ -1,0 +1,175 @@
+// fwd_kernel.cuh -- forward of the SiLU-gated RMSNorm on sm_100a.
+//
+// y = x * rsqrt(mean(x^2) + eps) * w * g * sigmoid(g) over packed BF16 rows [M, N]; the
+// FP32 rstd of every row is saved for the backward.  (flashinfer PR #8701, "perf(
+// cake_rmsnorm_silu_gate_train): L2-prefetching extra-long forward on SM107": the forward
+// of "Cake's SiLU-gated RMSNorm training kernel"; the pages print no kernel, so the design
+// below is this library's own.)
+//
+// Design: a persistent, warp-specialised CTA.  Warp 0 (one elected lane) streams row
+// blocks of x and g from HBM into a ring of shared-memory stages with 1-D TMA bulk copies
+// (rows are packed, so a block of R rows of one tensor is one contiguous copy) and
+// mbarrier transaction counts.  The consumer warps own `TPR` threads per row and `CPT`
+// 16-byte chunks per thread: pass 1 reads x from shared memory and reduces the sum of
+// squares (shuffles, plus named-barrier slots when a row spans several warps); pass 2
+// reads g and writes y straight to HBM with 16-byte stores.  Row blocks are assigned
+// round-robin (block b, b + grid, ...), a pure function of the launch plan.
+#pragma once
+
+#include "args.h"
+#include "device_common.cuh"
+
+namespace gnorm {
+
+
+template <int TPR, int CPT>
+__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
+    gated_rmsnorm_fwd_kernel(const FwdArgs a) {
+  constexpr int kNCT = consumer_threads_for(TPR);
+  constexpr int kGroups = kNCT / TPR;
+  extern __shared__ __align__(128) uint8_t smem[];
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+  uint64_t* empty = full + kMaxStages;
+  long long* blk_id = reinterpret_cast<long long*>(smem + 256);
+  float* red_slots = reinterpret_cast<float*>(smem + kRedSlotOffset);
+  uint8_t* stage0 = smem + kHeaderBytes;
+
+  const int S = a.stages;
+  const int R = a.rows_per_stage;
+  const int N = a.N;
+  const uint32_t tensor_bytes = static_cast<uint32_t>(R) * N * 2u;  // one tensor of a stage
+  const uint32_t stage_bytes = (2u * tensor_bytes + 127u) & ~127u;
+  constexpr int num_consumer_warps = kNCT / 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], num_consumer_warps);
+    }
+    fence_barrier_init();
+  }
+  __syncthreads();
+  grid_dependency_wait();     // inputs may come from the previous kernel on the stream
+  allow_dependent_launch();   // the next kernel may start its prologue on free SMs
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (warp == 0) {
+    // ---------------- producer: one lane issues the bulk copies ----------------
+    if (lane == 0) {
+      int s = 0;
+      uint32_t phase = 0;
+      for (long long blk = blockIdx.x;; blk += gridDim.x) {
+        if (!mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty)) break;
+        if (blk >= a.num_blocks) {
+          blk_id[s] = -1;
+          mbar_arrive(&full[s]);
+          break;
+        }
+        blk_id[s] = blk;
+        const long long r0 = blk * R;
+        const long long left = a.M - r0;
+        const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
+        const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+        uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
+        mbar_arrive_expect_tx(&full[s], 2u * bytes);
+        bulk_copy_g2s(st, a.x + r0 * N, bytes, &full[s]);
+        bulk_copy_g2s(st + tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+        if (++s == S) {
+          s = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int ctid = threadIdx.x - 32;
+  const int group = ctid / TPR;         // row slot inside a pass over the stage
+  const int lr = ctid - group * TPR;    // thread index inside the row
+  const int n8 = N >> 3;                // 16-byte chunks per row
+
+  float wf[CPT][8];
+  bool cval[CPT];
+#pragma unroll
+  for (int k = 0; k < CPT; ++k) {
+    const int c = k * TPR + lr;
+    cval[k] = c < n8;
+    if (cval[k]) {
+      const uint4 wv = *reinterpret_cast<const uint4*>(a.w + c * 8);
+      bf16x8_to_f32(wv, wf[k]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) wf[k][e] = 0.f;
+    }
+  }
+
+  int s = 0;
+  uint32_t phase = 0;
+  int slot = 0;
+  while (true) {
+    if (!mbar_wait(&full[s], phase, a.err, kErrWaitFull)) break;
+    const long long blk = blk_id[s];
+    if (blk < 0) break;
+    const long long r0 = blk * R;
+    const long long left = a.M - r0;
+    const int rows = static_cast<int>(left < R ? left : R);
+    const uint8_t* sx = stage0 + static_cast<size_t>(s) * stage_bytes;
+    const uint8_t* sg = sx + tensor_bytes;
+
+    for (int rb = 0; rb < rows; rb += kGroups) {
+      const int row = rb + group;
+      const bool valid = row < rows;
+      const int srow = valid ? row : 0;  // keep shared-memory reads inside the stage
+      const size_t roff = static_cast<size_t>(srow) * N * 2;
+
+      // pass 1: sum of squares of the row
+      uint4 xv[CPT];
+      float ss = 0.f;
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        if (cval[k]) {
+          xv[k] = *reinterpret_cast<const uint4*>(sx + roff + (k * TPR + lr) * 16);
+          float f[8];
+          bf16x8_to_f32(xv[k], f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+        }
+      }
+      ss = row_sum<TPR>(ss, red_slots, group, lr, slot);
+      slot ^= 1;
+      const float r = rsqrtf(fmaf(ss, a.inv_n, a.eps));
+      const long long grow = r0 + row;
+      if (valid && lr == 0) a.rstd[grow] = r;
+
+      // pass 2: y = xhat * w * g * sigmoid(g)
+#pragma unroll
+      for (int k = 0; k < CPT; ++k) {
+        if (cval[k]) {
+          const int c = k * TPR + lr;
+          const uint4 gv = *reinterpret_cast<const uint4*>(sg + roff + c * 16);
+          float xf[8], gf[8], yf[8];
+          bf16x8_to_f32(xv[k], xf);
+          bf16x8_to_f32(gv, gf);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float silu = gf[e] * sigmoid_f32(gf[e]);
+            yf[e] = ((xf[e] * r) * wf[k][e]) * silu;
+          }
+          if (valid)
+            *reinterpret_cast<uint4*>(a.y + grow * N + c * 8) = f32x8_to_bf16(yf);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (++s == S) {
+      s = 0;
+      phase ^= 1u;
+    }
+  }
+}
+
+}  // namespace gnorm

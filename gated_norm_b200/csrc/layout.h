@@ -1,0 +1,24 @@
+// layout.h -- constants shared by the host-side plan and the kernels.
+#pragma once
+
+#ifdef __CUDACC__
+#define GNORM_HD __host__ __device__
+#else
+#define GNORM_HD
+#endif
+
+namespace gnorm {
+
+constexpr int kMaxStages = 16;       // mbarrier pairs reserved in the shared-memory header
+constexpr int kHeaderBytes = 1024;   // barriers, block ids, flags and reduction slots
+constexpr int kRedSlotOffset = 512;  // float slots for cross-warp row reductions
+constexpr int kWorkspaceHeader = 256;  // workspace bytes before the dw partials
+constexpr int kReduceThreads = 512;  // dw second pass: 16 partial lanes x 32 column quads
+
+// Computing threads per CTA for a row geometry: 8 warps, or one 16-warp row group for the
+// widest rows.  One more warp (the producer) issues the copies.
+GNORM_HD constexpr int consumer_threads_for(int threads_per_row) {
+  return threads_per_row > 256 ? threads_per_row : 256;
+}
+
+}  // namespace gnorm

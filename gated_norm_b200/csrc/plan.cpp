@@ -1,0 +1,131 @@
+// plan.cpp -- the rows-per-SM dispatch rule (pure host code; needs no GPU).
+//
+// flashinfer PR #8701 ("perf(cake_rmsnorm_silu_gate_train): L2-prefetching extra-long
+// forward on SM107", PR description and commit message) routes its forward by architecture
+// and by rows per SM (M / #SMs) into "long" and "extra-long" tiers with per-architecture
+// thresholds.  This rule is this library's own for B200: it picks a row geometry from N,
+// then sizes the pipeline stage from the bytes one row brings in, and splits the rows
+// evenly over one persistent CTA per SM.  The tiers are:
+//   rows per SM <= the stage's target rows : one block per CTA (latency tier, small M);
+//   otherwise                              : k blocks per CTA, block size chosen so all
+//                                            CTAs get the same number of rows (streaming).
+#include <algorithm>
+#include <cstdint>
+#include <cstring>
+
+#include "gnorm.h"
+#include "layout.h"
+#include "plan.h"
+
+namespace gnorm {
+
+static TuningKnobs g_knobs;  // all zero: built-in values
+
+void set_tuning(const TuningKnobs& k) { g_knobs = k; }
+TuningKnobs get_tuning() { return g_knobs; }
+
+RowGeometry geometry_for(int64_t N) {
+  const int64_t n8 = N / 8;
+  if (n8 <= 4) return {4, 1};
+  if (n8 <= 8) return {8, 1};
+  if (n8 <= 16) return {16, 1};
+  if (n8 <= 32) return {32, 1};
+  if (n8 <= 64) return {32, 2};
+  if (n8 <= 128) return {32, 4};
+  if (n8 <= 256) return {64, 4};
+  if (n8 <= 512) return {128, 4};
+  if (n8 <= 1024) return {256, 4};
+  return {512, 4};
+}
+
+static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
+              int smem_per_block, gnorm_plan* out) {
+  if (out == nullptr) return GNORM_ERR_NULL;
+  std::memset(out, 0, sizeof(*out));
+  if (kind != 0 && kind != 1) return GNORM_ERR_ARG;
+  if (M < 0 || N < 8 || N > GNORM_N_MAX || (N % 8) != 0) return GNORM_ERR_SHAPE;
+  if (num_sms <= 0) return GNORM_ERR_ARG;
+  if (smem_per_block <= 0) smem_per_block = kB200SmemPerBlock;
+
+  const RowGeometry geo = geometry_for(N);
+  const int nct = consumer_threads_for(geo.threads_per_row);
+  const int groups = nct / geo.threads_per_row;
+  const int tensors = kind == 0 ? 2 : 3;
+  const int64_t row_bytes = static_cast<int64_t>(tensors) * N * 2;
+
+  const int ctas_per_sm = g_knobs.ctas_per_sm > 0 ? g_knobs.ctas_per_sm : 1;
+  const int64_t stage_target = g_knobs.stage_bytes > 0 ? g_knobs.stage_bytes : kStageTargetBytes;
+  const int max_stages =
+      std::min(kMaxStages, g_knobs.max_stages > 0 ? g_knobs.max_stages : kMaxStages);
+
+  // Shared memory available to one CTA when `ctas_per_sm` share an SM.
+  int64_t smem_cta = smem_per_block;
+  if (ctas_per_sm > 1)
+    smem_cta = std::min<int64_t>(smem_cta, kB200SmemPerSm / ctas_per_sm - kSmemPerCtaReserve);
+  const int64_t budget = smem_cta - kHeaderBytes;
+
+  // Rows per stage: about `stage_target` bytes, at least one row per row group.
+  int64_t target_rows = std::max<int64_t>(groups, stage_target / row_bytes);
+  while (target_rows > 1 && 2 * target_rows * row_bytes > budget) --target_rows;
+  if (2 * row_bytes > budget) return GNORM_ERR_UNSUPPORTED;  // two stages of one row
+
+  const int64_t grid_max = static_cast<int64_t>(num_sms) * ctas_per_sm;
+  int64_t R, blocks, grid;
+  if (M == 0) {
+    R = target_rows;
+    blocks = 0;
+    grid = 0;
+  } else {
+    const int64_t rows_per_cta = ceil_div(M, grid_max);
+    if (rows_per_cta <= target_rows) {
+      R = rows_per_cta;  // latency tier: one block per CTA
+    } else {
+      const int64_t k = ceil_div(rows_per_cta, target_rows);
+      R = ceil_div(rows_per_cta, k);  // streaming tier: k equal blocks per CTA
+    }
+    blocks = ceil_div(M, R);
+    grid = std::min(blocks, grid_max);
+  }
+
+  const int64_t stage_bytes = (static_cast<int64_t>(tensors) * R * N * 2 + 127) / 128 * 128;
+  int64_t stages = std::min<int64_t>(max_stages, budget / stage_bytes);
+  if (stages < 2) return GNORM_ERR_UNSUPPORTED;
+
+  // The backward reuses the stage buffers at the end for the per-group dw rows and, in the
+  // fused tail, for the reduction scratch.
+  int64_t body = stages * stage_bytes;
+  if (kind == 1) body = std::max<int64_t>(body, static_cast<int64_t>(groups) * N * 4 + nct * 16);
+  const int64_t smem = kHeaderBytes + body;
+  if (smem > smem_cta) return GNORM_ERR_UNSUPPORTED;
+
+  out->kind = kind;
+  out->threads_per_row = geo.threads_per_row;
+  out->chunks_per_thread = geo.chunks_per_thread;
+  out->consumer_threads = nct;
+  out->rows_per_stage = static_cast<int>(R);
+  out->stages = static_cast<int>(stages);
+  out->ctas_per_sm = ctas_per_sm;
+  out->grid = static_cast<int>(grid);
+  out->num_blocks = blocks;
+  out->smem_bytes = static_cast<int>(smem);
+  if (kind == 1) {
+    out->dynamic_schedule = deterministic ? 0 : 1;
+    out->partials = static_cast<int>(grid);
+    // The last-CTA tail pays off when the partials are small; wide rows use the second
+    // launch, whose CTAs read the partials in parallel.
+    out->fused_reduce =
+        (!deterministic && grid > 0 && static_cast<int64_t>(grid) * N <= kFusedReduceMaxFloats)
+            ? 1
+            : 0;
+  }
+  return GNORM_OK;
+}
+
+size_t workspace_bytes_for(const gnorm_plan& p, int64_t N) {
+  const size_t raw = kWorkspaceHeader + static_cast<size_t>(p.partials) * N * 4;
+  return (raw + GNORM_WORKSPACE_ALIGN - 1) / GNORM_WORKSPACE_ALIGN * GNORM_WORKSPACE_ALIGN;
+}
+
+}  // namespace gnorm

@@ -1,0 +1,228 @@
+"""Python binding of libgnorm: the same entry points as include/gnorm.h.
+
+Argument marshalling only.  Tensors are torch CUDA tensors (torch provides device memory
+and streams); every step of the computation runs in the library's CUDA kernels.  Outputs
+that are not passed in are allocated with ``torch.empty``; errors reported by the library
+raise ``GnormError``.
+"""
+from __future__ import annotations
+
+import ctypes
+import threading
+
+import torch
+
+from ._lib import GNORM_OK, GnormPlan, lib
+
+__all__ = [
+    "GnormError",
+    "gnorm_fwd",
+    "gnorm_bwd",
+    "gnorm_ckpt_step",
+    "gnorm_bwd_workspace_bytes",
+    "gnorm_bwd_workspace_bytes_for",
+    "gnorm_status_string",
+    "gnorm_plan_query",
+    "gnorm_device_error",
+    "gnorm_set_tuning",
+    "gnorm_build_info",
+    "workspace",
+]
+
+
+class GnormError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {gnorm_status_string(status)} (status {status})")
+
+
+def gnorm_status_string(status: int) -> str:
+    return lib.gnorm_status_string(int(status)).decode()
+
+
+def gnorm_build_info() -> str:
+    return lib.gnorm_build_info().decode()
+
+
+def gnorm_bwd_workspace_bytes(M: int, N: int, deterministic: bool = True) -> int:
+    return int(lib.gnorm_bwd_workspace_bytes(int(M), int(N), int(bool(deterministic))))
+
+
+def gnorm_bwd_workspace_bytes_for(M: int, N: int, deterministic: bool, num_sms: int) -> int:
+    return int(lib.gnorm_bwd_workspace_bytes_for(int(M), int(N), int(bool(deterministic)),
+                                                 int(num_sms)))
+
+
+def gnorm_plan_query(kind: int, M: int, N: int, deterministic: bool, num_sms: int,
+                     smem_per_block: int = 0) -> dict:
+    """The dispatch rule for `kind` (0 fwd, 1 bwd) on a device with `num_sms` SMs."""
+    p = GnormPlan()
+    st = lib.gnorm_plan_query(int(kind), int(M), int(N), int(bool(deterministic)), int(num_sms),
+                              int(smem_per_block), ctypes.byref(p))
+    if st != GNORM_OK:
+        raise GnormError(st, "gnorm_plan_query")
+    return p.as_dict()
+
+
+def gnorm_device_error(reset: bool = False) -> int:
+    return int(lib.gnorm_device_error(int(bool(reset))))
+
+
+def gnorm_set_tuning(stage_bytes: int = 0, max_stages: int = 0, ctas_per_sm: int = 0,
+                     disable_pdl: bool = False) -> None:
+    lib.gnorm_set_tuning(int(stage_bytes), int(max_stages), int(ctas_per_sm),
+                         int(bool(disable_pdl)))
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr() if t.numel() else 0)
+
+
+def _stream(stream, device) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _rows(t: torch.Tensor, name: str):
+    if t.dim() < 1:
+        raise ValueError(f"{name} must have a last dimension N")
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (packed rows)")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    N = t.shape[-1]
+    return t.numel() // N if N else 0, N
+
+
+def _same(a: torch.Tensor, b: torch.Tensor, an: str, bn: str):
+    if a.shape != b.shape:
+        raise ValueError(f"{an} {tuple(a.shape)} and {bn} {tuple(b.shape)} differ")
+    if a.device != b.device:
+        raise ValueError(f"{an} and {bn} are on different devices")
+
+
+def _vec(t: torch.Tensor, N: int, dtypes, name: str, device):
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} must be one of {dtypes}, got {t.dtype}")
+    if t.numel() != N or not t.is_contiguous() or t.device != device:
+        raise ValueError(f"{name} must be a contiguous [{N}] tensor on {device}")
+
+
+def _check(st: int, where: str):
+    if st != GNORM_OK:
+        raise GnormError(st, where)
+
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def workspace(M: int, N: int, deterministic: bool, device) -> torch.Tensor:
+    """A zero-initialised backward workspace for `device`, cached and grown as needed.
+
+    The cache holds one buffer per device; calls that may run concurrently (other streams)
+    must pass workspaces of their own.
+    """
+    device = torch.device(device)
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    with torch.cuda.device(idx):
+        need = max(gnorm_bwd_workspace_bytes(M, N, deterministic), 256)
+    with _ws_lock:
+        buf = _ws_cache.get(idx)
+        if buf is None or buf.numel() < need:
+            buf = torch.zeros(need, dtype=torch.uint8, device=torch.device("cuda", idx))
+            _ws_cache[idx] = buf
+        return buf
+
+
+# ------------------------------------------------------------------------- entry points
+
+def gnorm_fwd(x, g, w, eps: float = 1e-6, *, y=None, rstd=None, stream=None):
+    """Forward: returns (y, rstd).  x, g: [..., N] BF16; w: [N] BF16; rstd: FP32 [M]."""
+    M, N = _rows(x, "x")
+    _rows(g, "g")
+    _same(x, g, "x", "g")
+    _vec(w, N, (torch.bfloat16,), "w", x.device)
+    if y is None:
+        y = torch.empty_like(x)
+    else:
+        _rows(y, "y")
+        _same(x, y, "x", "y")
+    if rstd is None:
+        rstd = torch.empty(M, dtype=torch.float32, device=x.device)
+    else:
+        _vec(rstd, M, (torch.float32,), "rstd", x.device)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_fwd(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(y), _ptr(rstd), M, N,
+                           _stream(stream, x.device))
+    _check(st, "gnorm_fwd")
+    return y, rstd
+
+
+def _bwd_outputs(x, N, dx, dg, dw, dw_fp32):
+    if dx is None:
+        dx = torch.empty_like(x)
+    else:
+        _rows(dx, "dx")
+        _same(x, dx, "x", "dx")
+    if dg is None:
+        dg = torch.empty_like(x)
+    else:
+        _rows(dg, "dg")
+        _same(x, dg, "x", "dg")
+    dw_dtype = torch.float32 if dw_fp32 else torch.bfloat16
+    if dw is None:
+        dw = torch.empty(N, dtype=dw_dtype, device=x.device)
+    else:
+        _vec(dw, N, (dw_dtype,), "dw", x.device)
+    return dx, dg, dw
+
+
+def gnorm_bwd(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: bool = False,
+              deterministic: bool = True, workspace_buf=None, stream=None):
+    """Backward: returns (dx, dg, dw).  dw is FP32 if dw_fp32 else BF16."""
+    M, N = _rows(x, "x")
+    for t, n in ((dy, "dy"), (g, "g")):
+        _rows(t, n)
+        _same(x, t, "x", n)
+    _vec(w, N, (torch.bfloat16,), "w", x.device)
+    _vec(rstd, M, (torch.float32,), "rstd", x.device)
+    dx, dg, dw = _bwd_outputs(x, N, dx, dg, dw, dw_fp32)
+    ws = workspace_buf if workspace_buf is not None else workspace(M, N, deterministic, x.device)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_bwd(_ptr(dy), _ptr(x), _ptr(g), _ptr(w), _ptr(rstd), _ptr(dx), _ptr(dg),
+                           _ptr(dw), int(bool(dw_fp32)), int(bool(deterministic)), M, N, _ptr(ws),
+                           ws.numel() * ws.element_size(), _stream(stream, x.device))
+    _check(st, "gnorm_bwd")
+    return dx, dg, dw
+
+
+def gnorm_ckpt_step(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=None, dw=None,
+                    dw_fp32: bool = False, deterministic: bool = True, workspace_buf=None,
+                    stream=None):
+    """Checkpointed step (forward, forward again, backward): returns (y, rstd, dx, dg, dw)."""
+    M, N = _rows(x, "x")
+    for t, n in ((dy, "dy"), (g, "g")):
+        _rows(t, n)
+        _same(x, t, "x", n)
+    _vec(w, N, (torch.bfloat16,), "w", x.device)
+    if y is None:
+        y = torch.empty_like(x)
+    if rstd is None:
+        rstd = torch.empty(M, dtype=torch.float32, device=x.device)
+    else:
+        _vec(rstd, M, (torch.float32,), "rstd", x.device)
+    dx, dg, dw = _bwd_outputs(x, N, dx, dg, dw, dw_fp32)
+    ws = workspace_buf if workspace_buf is not None else workspace(M, N, deterministic, x.device)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_ckpt_step(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(dy), _ptr(y),
+                                 _ptr(rstd), _ptr(dx), _ptr(dg), _ptr(dw), int(bool(dw_fp32)),
+                                 int(bool(deterministic)), M, N, _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream, x.device))
+    _check(st, "gnorm_ckpt_step")
+    return y, rstd, dx, dg, dw

@@ -1,0 +1,177 @@
+/*
+ * gnorm.h -- C ABI of libgnorm: SiLU-gated RMSNorm training kernels for B200 (sm_100a).
+ *
+ * The operation is "Cake's SiLU-gated RMSNorm training kernel" of flashinfer PR #8701
+ * ("perf(cake_rmsnorm_silu_gate_train): L2-prefetching extra-long forward on SM107",
+ * PR description), with the semantics of the comparator kernels listed in that page's
+ * section "How the tables were measured" (FLA rms_norm_gated, mamba_ssm rmsnorm_fn):
+ * normalise each row, scale by the weight, gate by silu(g).  For a row x of length N,
+ * gate g, weight w and upstream gradient dy:
+ *
+ *     r   = 1 / sqrt(mean_j(x_j^2) + eps)                      (rstd, FP32, saved)
+ *     y_j = x_j * r * w_j * g_j * sigmoid(g_j)                 (BF16)
+ *     xhat = x r,  s = g sigmoid(g),  u = dy w s,  c = mean_j(u_j xhat_j)
+ *     dx  = r (u - xhat c)                                     (BF16)
+ *     dg  = dy xhat w sigmoid(g) (1 + g (1 - sigmoid(g)))      (BF16)
+ *     dw  = sum over rows of dy xhat s                         (BF16 or FP32)
+ *
+ * Conventions for every entry point:
+ *   - Tensors are row-major and contiguous ("packed" rows): element (m, j) of an [M, N]
+ *     tensor sits at index m*N + j.  x, g, w, y, dy, dx, dg are BF16 (IEEE bfloat16 bit
+ *     patterns, 2 bytes); rstd is FP32; dw is BF16 or FP32 (dw_fp32).
+ *   - All tensor pointers are DEVICE pointers of the current CUDA device.  Every pointer
+ *     except rstd must be 16-byte aligned; rstd must be 4-byte aligned.
+ *   - N must be a multiple of 8 with 8 <= N <= GNORM_N_MAX.  M >= 0; M == 0 is a no-op
+ *     for the forward, and the backward then writes dw = 0.  When M == 0 the per-row
+ *     tensors may be NULL.
+ *   - eps must be finite and >= 0.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only enqueue
+ *     work: they never synchronise, never allocate and are safe to capture in a CUDA
+ *     graph.  Each call is launched with programmatic dependent launch, so a kernel of
+ *     this library may start its prologue while the previous kernel on the stream drains;
+ *     it reads and writes global memory only after that kernel has completed.
+ *   - The caller owns every buffer; the library keeps no pointer after a call returns.
+ *   - Outputs must not overlap any input or each other (GNORM_ERR_ALIAS).
+ *   - Errors are detected on the host before any launch and returned as a gnorm_status;
+ *     no kernel traps.  A CUDA error at launch returns GNORM_ERR_CUDA.
+ */
+#ifndef GNORM_H_
+#define GNORM_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define GNORM_API __attribute__((visibility("default")))
+#else
+#define GNORM_API
+#endif
+
+#define GNORM_N_MAX 16384
+#define GNORM_WORKSPACE_ALIGN 256
+
+typedef enum gnorm_status {
+  GNORM_OK = 0,
+  GNORM_ERR_NULL = -1,        /* a required pointer is NULL */
+  GNORM_ERR_SHAPE = -2,       /* M < 0, N not a multiple of 8, N < 8 or N > GNORM_N_MAX */
+  GNORM_ERR_ALIGN = -3,       /* a pointer breaks the alignment rule above */
+  GNORM_ERR_ALIAS = -4,       /* an output overlaps an input or another output */
+  GNORM_ERR_UNSUPPORTED = -5, /* no kernel plan fits the device (e.g. too little shared memory) */
+  GNORM_ERR_WORKSPACE = -6,   /* workspace NULL, misaligned or smaller than required */
+  GNORM_ERR_CUDA = -7,        /* the CUDA runtime reported an error */
+  GNORM_ERR_ARG = -8          /* another argument is out of range (eps, flags, kind) */
+} gnorm_status;
+
+/*
+ * Forward.  Reads x[M,N], g[M,N], w[N]; writes y[M,N] (BF16) and rstd[M] (FP32).
+ * Flashinfer PR #8701, section "How the tables were measured": "fwd" is one forward call.
+ * The result does not depend on any mode flag: the deterministic and non-deterministic
+ * packages of that page produce bitwise-equal y (commit message of the PR).
+ */
+GNORM_API int gnorm_fwd(const void* x, const void* g, const void* w, float eps,
+              void* y, float* rstd, int64_t M, int64_t N, void* stream);
+
+/*
+ * Backward.  Reads dy, x, g [M,N], w[N] and the forward's rstd[M]; writes dx, dg [M,N]
+ * (BF16) and dw[N] (BF16 if dw_fp32 == 0, else FP32).  dw is overwritten, not accumulated.
+ * Flashinfer PR #8701, section "How the tables were measured": "bwdg" (BF16 dw) and
+ * "bwdg_f32" (FP32 dw); the deterministic package is the same API with deterministic=True.
+ *
+ * deterministic != 0: rows are assigned to CTAs by a fixed rule and the FP32 dw partials are
+ *   summed in a fixed order by a second launch, so dx, dg and dw are bitwise identical from
+ *   run to run on the same device model with the same arguments.
+ * deterministic == 0: CTAs take row blocks from a shared counter, so dw's FP32 summation
+ *   order can change between runs (dx and dg do not); dw is never accumulated with float
+ *   atomics.
+ *
+ * workspace: device scratch of at least gnorm_bwd_workspace_bytes(M, N, deterministic)
+ *   bytes, GNORM_WORKSPACE_ALIGN-aligned.  Its first GNORM_WORKSPACE_ALIGN bytes must be
+ *   zero before the first call (e.g. cudaMemset once after allocation); every call leaves
+ *   them zero again.  Concurrent calls must not share a workspace.
+ */
+GNORM_API int gnorm_bwd(const void* dy, const void* x, const void* g, const void* w, const float* rstd,
+              void* dx, void* dg, void* dw, int dw_fp32, int deterministic,
+              int64_t M, int64_t N, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Checkpointed training step: forward, forward again (activation recomputation), backward,
+ * all enqueued on `stream`.  Flashinfer PR #8701, section "How the tables were measured":
+ * "ckptg" is the checkpointed step (2 x forward + backward), "stepg_f32" the same with an
+ * FP32 dw.  y and rstd hold the second forward's outputs (bitwise equal to the first's);
+ * the backward consumes that rstd.  Arguments as for gnorm_fwd and gnorm_bwd.
+ */
+GNORM_API int gnorm_ckpt_step(const void* x, const void* g, const void* w, float eps, const void* dy,
+                    void* y, float* rstd, void* dx, void* dg, void* dw,
+                    int dw_fp32, int deterministic, int64_t M, int64_t N,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Workspace bytes gnorm_bwd / gnorm_ckpt_step need on the CURRENT device (reads its SM count).
+ * Returns 0 if the arguments are invalid or no device is present.
+ */
+GNORM_API size_t gnorm_bwd_workspace_bytes(int64_t M, int64_t N, int deterministic);
+
+/* The same for a device with `num_sms` SMs.  Pure host function; needs no GPU. */
+GNORM_API size_t gnorm_bwd_workspace_bytes_for(int64_t M, int64_t N, int deterministic, int num_sms);
+
+/* Human-readable name of a gnorm_status value (static storage). */
+GNORM_API const char* gnorm_status_string(int status);
+
+/*
+ * Launch plan chosen by the rows-per-SM dispatch rule.  Flashinfer PR #8701 (PR description
+ * and commit message) routes its forward by architecture and by rows per SM
+ * (M / number of SMs) into tiers; this library's rule is its own, tuned for B200.
+ */
+typedef struct gnorm_plan {
+  int kind;              /* 0 forward, 1 backward */
+  int threads_per_row;   /* threads that share one row */
+  int chunks_per_thread; /* 16-byte chunks (8 BF16 values) per thread and tensor */
+  int consumer_threads;  /* computing threads per CTA (one extra warp issues the copies) */
+  int rows_per_stage;    /* rows copied into shared memory per pipeline stage */
+  int stages;            /* pipeline depth */
+  int ctas_per_sm;       /* resident CTAs per SM */
+  int grid;              /* persistent CTAs launched */
+  int64_t num_blocks;    /* row blocks: ceil(M / rows_per_stage) */
+  int smem_bytes;        /* dynamic shared memory per CTA */
+  int dynamic_schedule;  /* 1: CTAs take row blocks from an atomic counter */
+  int fused_reduce;      /* 1: the last CTA to finish reduces the dw partials */
+  int partials;          /* rows of the FP32 dw partial buffer (backward), else 0 */
+  int reserved;
+} gnorm_plan;
+
+/*
+ * The dispatch rule as a pure host function: plan for `kind` (0 fwd, 1 bwd) on a device with
+ * `num_sms` SMs and `smem_per_block` bytes of opt-in shared memory per CTA (0 = 232448, the
+ * B200 value).  Needs no GPU.  Returns GNORM_OK or an error status.
+ */
+GNORM_API int gnorm_plan_query(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
+                     int smem_per_block, gnorm_plan* out);
+
+/*
+ * Device-side error word: kernels set a bit here if a bounded wait inside them gave up
+ * (1 = a wait for copied data, 2 = a wait for a free pipeline stage).  Synchronises the
+ * current device, returns the word and clears it if `reset` != 0.  Returns -1 (as an int)
+ * if the word cannot be read.
+ */
+GNORM_API int gnorm_device_error(int reset);
+
+/*
+ * Process-wide tuning knobs for experiments (0 keeps the built-in value): target bytes per
+ * pipeline stage, maximum pipeline depth, resident CTAs per SM, and 1 to launch without
+ * programmatic dependent launch.  Affects plans made after the call, including
+ * gnorm_plan_query and gnorm_bwd_workspace_bytes.  Not thread-safe with concurrent calls.
+ */
+GNORM_API void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl);
+
+/* Build description: compiler version, target architecture (static storage). */
+GNORM_API const char* gnorm_build_info(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GNORM_H_ */
