@@ -37,3 +37,9 @@ def test_dw_and_rstd_rules():
     assert not dw_fp32_check(ref * (1 + 5e-3), ref)["ok"]
     assert rstd_check(ref[[0, 1, 3]] * (1 + 5e-6), ref[[0, 1, 3]])["ok"]
     assert not rstd_check(ref[[0, 1, 3]] * (1 + 5e-5), ref[[0, 1, 3]])["ok"]
+
+
+def test_subnormal_results_may_flush_to_zero():
+    ref = np.array([[1e-40, -3e-39, 0.0]])
+    assert bf16_check(np.zeros_like(ref), ref)["ok"]
+    assert not bf16_check(np.array([[1e-37, 0.0, 0.0]]), ref)["ok"]
