@@ -2,12 +2,13 @@
 
 The kernels live in ``libgnorm.so`` behind the C ABI of ``include/gnorm.h``; this package
 is a thin binding over it.  Importing the package loads the library and fails loudly if it
-has not been built (``python -m gated_norm_b200.build``): there is no CPU fallback.
+has not been built (``python gated_norm_b200/build.py``): there is no CPU fallback.
 """
 from .gnorm import (  # noqa: F401
     GnormError,
     gnorm_build_info,
     gnorm_bwd,
+    gnorm_bwd_noalloc,
     gnorm_bwd_workspace_bytes,
     gnorm_bwd_workspace_bytes_for,
     gnorm_ckpt_step,

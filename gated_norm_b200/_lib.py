@@ -1,6 +1,6 @@
 """ctypes loader for libgnorm.so (the C ABI declared in include/gnorm.h).
 
-The shared library is built in-tree (``python -m gated_norm_b200.build``).  There is no
+The shared library is built in-tree (``python gated_norm_b200/build.py``).  There is no
 fallback: if the library is missing, importing this module raises.
 """
 from __future__ import annotations
@@ -58,6 +58,8 @@ SIGNATURES = {
     "gnorm_fwd": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _i64, _i64, _vp]),
     "gnorm_bwd": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64, _vp, _sz,
                          _vp]),
+    "gnorm_bwd_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64,
+                                 _vp]),
     "gnorm_ckpt_step": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
                                _i64, _vp, _sz, _vp]),
     "gnorm_bwd_workspace_bytes": (_sz, [_i64, _i64, _int]),
@@ -73,7 +75,7 @@ SIGNATURES = {
 def load(path: str = LIB_PATH) -> ctypes.CDLL:
     if not os.path.exists(path):
         raise ImportError(
-            f"{path} is missing: build it with `python -m gated_norm_b200.build` "
+            f"{path} is missing: build it with `python gated_norm_b200/build.py` "
             "(the CUDA path has no CPU fallback)")
     lib = ctypes.CDLL(path)
     for name, (res, args) in SIGNATURES.items():

@@ -1,6 +1,8 @@
 """Build libgnorm.so in-tree with nvcc for sm_100a.
 
-    python -m gated_norm_b200.build [--force] [--verbose]
+    python gated_norm_b200/build.py [--force] [--verbose]
+
+(run it as a script: importing the package loads the library, which this script makes)
 
 Each source is compiled to an object under ``<repo>/_build/`` (in parallel), then linked
 into ``gated_norm_b200/libgnorm.so``.  The CUDA runtime is linked statically and its
@@ -26,7 +28,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgnorm.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "plan.cpp"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "plan.cpp", "noalloc.cu"]
 
 
 def nvcc() -> str:

@@ -19,6 +19,7 @@ __all__ = [
     "gnorm_fwd",
     "gnorm_bwd",
     "gnorm_ckpt_step",
+    "gnorm_bwd_noalloc",
     "gnorm_bwd_workspace_bytes",
     "gnorm_bwd_workspace_bytes_for",
     "gnorm_status_string",
@@ -199,6 +200,28 @@ def gnorm_bwd(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: bool = F
                            _ptr(dw), int(bool(dw_fp32)), int(bool(deterministic)), M, N, _ptr(ws),
                            ws.numel() * ws.element_size(), _stream(stream, x.device))
     _check(st, "gnorm_bwd")
+    return dx, dg, dw
+
+
+def gnorm_bwd_noalloc(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: bool = False,
+                      deterministic: bool = True, stream=None):
+    """Backward with the library's static scratch instead of a workspace.
+
+    For callers that cannot allocate device memory.  Calls that overlap on the GPU share
+    the scratch and race; see include/gnorm.h.
+    """
+    M, N = _rows(x, "x")
+    for t, n in ((dy, "dy"), (g, "g")):
+        _rows(t, n)
+        _same(x, t, "x", n)
+    _vec(w, N, (torch.bfloat16,), "w", x.device)
+    _vec(rstd, M, (torch.float32,), "rstd", x.device)
+    dx, dg, dw = _bwd_outputs(x, N, dx, dg, dw, dw_fp32)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_bwd_noalloc(_ptr(dy), _ptr(x), _ptr(g), _ptr(w), _ptr(rstd), _ptr(dx),
+                                   _ptr(dg), _ptr(dw), int(bool(dw_fp32)),
+                                   int(bool(deterministic)), M, N, _stream(stream, x.device))
+    _check(st, "gnorm_bwd_noalloc")
     return dx, dg, dw
 
 

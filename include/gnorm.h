@@ -98,6 +98,28 @@ GNORM_API int gnorm_bwd(const void* dy, const void* x, const void* g, const void
               int64_t M, int64_t N, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward without any caller-provided scratch (the pages have no counterpart to this entry
+ * point).  For callers that cannot allocate device memory -- a runtime whose device memory
+ * is owned up front by another allocator, a latency-critical loop that must not hit
+ * cudaMalloc's implicit synchronisation, a plug-in that only receives tensors -- and so
+ * cannot provide gnorm_bwd's workspace.  Same arguments and results as gnorm_bwd, minus the
+ * workspace; it allocates nothing and calls no allocating routine.
+ *
+ * Its scratch is a file-scope static device array of 4 MiB in the library, held on every
+ * GPU that loads the library until the process exits.  Calls whose FP32 dw partials need
+ * more (about partials x N x 4 bytes + 256; e.g. N > 7000 on a 148-SM B200) return
+ * GNORM_ERR_UNSUPPORTED.  The first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call before any stream
+ * capture.  Every call clears the array's 256-byte counter header on `stream` before its
+ * kernels start; all calls share the array, so calls that overlap on the GPU (other
+ * streams, other threads) race and must be serialised by the caller.  A wait timeout inside
+ * these kernels is recorded in the array's header, not in gnorm_device_error's word.
+ */
+GNORM_API int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, const void* w,
+                                const float* rstd, void* dx, void* dg, void* dw, int dw_fp32,
+                                int deterministic, int64_t M, int64_t N, void* stream);
+
+/*
  * Checkpointed training step: forward, forward again (activation recomputation), backward,
  * all enqueued on `stream`.  Flashinfer PR #8701, section "How the tables were measured":
  * "ckptg" is the checkpointed step (2 x forward + backward), "stepg_f32" the same with an
