@@ -5,10 +5,13 @@
 
 A step is one checkpointed training step over one batch of seeded synthetic rows:
 forward, forward again (recompute), backward with the dw reduction -- every stage of the
-path.  The default workload is 65536 x 128 (a per-head gated norm of a linear-attention
-output, 512 heads x 128 tokens).  Times are CUDA-event device times on the launching
-stream; L2 is flushed (256 MiB write) between steps and the flush is outside the timed
-events.  `value` is algorithmic HBM bytes of the whole job / max-over-ranks time (GB/s).
+path -- replayed from one CUDA graph ("ckptg").  Each timed step also replays the backward
+("bwdg") and the forward ("fwdg") alone, each from its own graph, for the per-operation
+times and the roofline of the dominant kernel.  The default workload is 65536 x 128 (a
+per-head gated norm of a linear-attention output, 512 heads x 128 tokens).  Times are
+CUDA-event device times on the launching stream; L2 is flushed (256 MiB write) before
+every timed replay, outside the events.  `value` is the checkpointed step's algorithmic
+HBM bytes of the whole job / the max-over-ranks summed step time (GB/s).
 
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the
 data path; the rows of a data-parallel batch are independent).  `--impl reference` times
@@ -61,6 +64,36 @@ def dist_env():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return rank, world, local
+
+
+def init_dist(device, backend="nccl"):
+    """One process per GPU; the process group's timeout bounds every collective."""
+    import datetime
+
+    import torch.distributed as dist
+
+    kwargs = {"timeout": datetime.timedelta(seconds=120)}
+    if backend == "nccl":
+        kwargs["device_id"] = device
+    dist.init_process_group(backend, **kwargs)
+    return dist
+
+
+def max_over_ranks(value, world, device):
+    """The largest value over all ranks (the job's time is its slowest rank's)."""
+    if world == 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbs(bytes_per_rank_step, steps, world, max_ms):
+    """Algorithmic bytes of all ranks' steps over the slowest rank's summed step time."""
+    return bytes_per_rank_step * steps * world / (max_ms * 1e-3) / 1e9
 
 
 def measured_peaks():
@@ -221,11 +254,7 @@ def run_ours(args, wl):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
+        dist = init_dist(dev, "nccl")
     import gated_norm_b200 as gn
 
     M, N, eps = wl.M, wl.N, wl.eps
@@ -244,32 +273,57 @@ def run_ours(args, wl):
                      device=dev)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    plan_b = gn.gnorm_plan_query(1, M, N, det, torch.cuda.get_device_properties(dev).
-                                 multi_processor_count)
-    launches_per_step = 2 + 1 + (0 if plan_b["fused_reduce"] else 1)
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    plan_b = gn.gnorm_plan_query(1, M, N, det, sms)
+    bwd_launches = 1 + (0 if plan_b["fused_reduce"] else 1)
+
+    # The operations as the pages time them: each replayed from its own CUDA graph.
+    def op_fwd():
+        gn.gnorm_fwd(x, g, w, eps, y=y, rstd=rstd)
+
+    def op_bwd():
+        gn.gnorm_bwd(dy, x, g, w, rstd, dx=dx, dg=dg, dw=dw, dw_fp32=fp32, deterministic=det,
+                     workspace_buf=ws)
+
+    def op_ckpt():
+        gn.gnorm_ckpt_step(x, g, w, eps, dy, y=y, rstd=rstd, dx=dx, dg=dg, dw=dw, dw_fp32=fp32,
+                           deterministic=det, workspace_buf=ws)
+
+    def capture(fn):
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+            fn()
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            fn()
+        return graph
+
+    graphs = {"ckpt": capture(op_ckpt), "bwd": capture(op_bwd), "fwd": capture(op_fwd)}
+    launches = {"ckpt": 2 + bwd_launches, "bwd": bwd_launches, "fwd": 1}
+    order = ("ckpt", "bwd", "fwd")
 
     def one_step(evs=None):
-        # the checkpointed step as its three entry points: forward, forward, backward
-        if evs:
-            evs[0].record(stream)
-        gn.gnorm_fwd(x, g, w, eps, y=y, rstd=rstd, stream=stream)
-        if evs:
-            evs[1].record(stream)
-        gn.gnorm_fwd(x, g, w, eps, y=y, rstd=rstd, stream=stream)
-        if evs:
-            evs[2].record(stream)
-        gn.gnorm_bwd(dy, x, g, w, rstd, dx=dx, dg=dg, dw=dw, dw_fp32=fp32, deterministic=det,
-                     workspace_buf=ws, stream=stream)
-        if evs:
-            evs[3].record(stream)
+        # one timed step: the checkpointed step (the measured unit), then the backward and
+        # the forward alone for the per-operation times; L2 is flushed before each, outside
+        # the events.
+        for j, name in enumerate(order):
+            flush.zero_()
+            if evs:
+                evs[2 * j].record(stream)
+            graphs[name].replay()
+            if evs:
+                evs[2 * j + 1].record(stream)
 
     for _ in range(args.warmup):
-        flush.zero_()
         one_step()
     torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
     clocks = ClockSampler(local)
     if rank == 0:
         clocks.start()
@@ -277,25 +331,18 @@ def run_ours(args, wl):
         dist.barrier()
     torch.cuda.synchronize()
     for i in range(K):
-        flush.zero_()
         one_step(evs[i])
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     clk = clocks.stop() if rank == 0 else None
 
-    t_fwd = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
-    t_fwd2 = [evs[i][1].elapsed_time(evs[i][2]) for i in range(K)]
+    t_ckpt = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
     t_bwd = [evs[i][2].elapsed_time(evs[i][3]) for i in range(K)]
-    t_step = [evs[i][0].elapsed_time(evs[i][3]) for i in range(K)]
-    total_ms = float(sum(t_step))
-    if world > 1:
-        tt = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms = float(tt.item())
-
+    t_fwd = [evs[i][4].elapsed_time(evs[i][5]) for i in range(K)]
+    total_ms = max_over_ranks(float(sum(t_ckpt)), world, dev)
     step_bytes = ckpt_bytes(M, N, fp32)
-    value = step_bytes * K * world / (total_ms * 1e-3) / 1e9
+    value = whole_job_gbs(step_bytes, K, world, total_ms)
     peak, peak_kind = measured_peaks()
 
     # one checkpointed step through the single public entry point, host buffers in and out
@@ -323,12 +370,8 @@ def run_ours(args, wl):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            tt = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            e_ms = float(tt.item())
-        e2e = {"value": step_bytes * args.e2e_steps * world / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": whole_job_gbs(step_bytes, args.e2e_steps, world, e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps,
                "path": "gnorm_ckpt_step with pinned host inputs copied in and outputs copied "
@@ -343,8 +386,7 @@ def run_ours(args, wl):
     def avg(v):
         return float(sum(v) / len(v))
 
-    us = {"fwd": avg(t_fwd) * 1e3, "fwd_recompute": avg(t_fwd2) * 1e3, "bwd": avg(t_bwd) * 1e3,
-          "ckpt": avg(t_step) * 1e3}
+    us = {"fwd": avg(t_fwd) * 1e3, "bwd": avg(t_bwd) * 1e3, "ckpt": avg(t_ckpt) * 1e3}
     gbs = {"fwd": fwd_bytes(M, N) / (us["fwd"] * 1e-6) / 1e9,
            "bwd": bwd_bytes(M, N, fp32) / (us["bwd"] * 1e-6) / 1e9,
            "ckpt": step_bytes / (us["ckpt"] * 1e-6) / 1e9}
@@ -361,21 +403,23 @@ def run_ours(args, wl):
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "M": M, "N": N, "eps": eps,
-                   "step": "checkpointed step: fwd, fwd (recompute), bwd + dw reduction",
+                   "step": "checkpointed step as one CUDA graph: fwd, fwd (recompute), bwd + dw reduction",
                    "deterministic": det, "dw": "fp32" if fp32 else "bf16",
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": f"dp{world} (independent rows per rank, no collective)"},
         "us_per_call": us,
+        "timing": "fwd, bwd, ckpt each replayed from its own CUDA graph (fwdg, bwdg, ckptg)",
         "gbs": gbs,
         "frac_of_peak": {k: v / peak for k, v in gbs.items()},
-        "roofline": {"bound": "hbm", "kernel": "gnorm_bwd (backward + dw second pass)",
+        "roofline": {"bound": "hbm", "kernel": "gnorm_bwd (backward kernel + dw second pass, "
+                                                "graph-replayed)",
                      "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
                      "frac": achieved / peak,
                      "algorithmic_bytes_per_launch": bwd_bytes(M, N, fp32),
                      "traffic": bwd_traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": sum(launches.values()) * K,
         "clocks": clk,
     }
     print(json.dumps(line))

@@ -13,6 +13,7 @@ from .gnorm import (  # noqa: F401
     gnorm_bwd_workspace_bytes_for,
     gnorm_ckpt_step,
     gnorm_device_error,
+    gnorm_dw_reduce,
     gnorm_fwd,
     gnorm_plan_query,
     gnorm_set_tuning,

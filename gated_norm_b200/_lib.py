@@ -62,12 +62,13 @@ SIGNATURES = {
                                  _vp]),
     "gnorm_ckpt_step": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
                                _i64, _vp, _sz, _vp]),
+    "gnorm_dw_reduce": (_int, [_vp, _i64, _i64, _vp, _int, _vp]),
     "gnorm_bwd_workspace_bytes": (_sz, [_i64, _i64, _int]),
     "gnorm_bwd_workspace_bytes_for": (_sz, [_i64, _i64, _int, _int]),
     "gnorm_status_string": (ctypes.c_char_p, [_int]),
     "gnorm_plan_query": (_int, [_int, _i64, _i64, _int, _int, _int, ctypes.POINTER(GnormPlan)]),
     "gnorm_device_error": (_int, [_int]),
-    "gnorm_set_tuning": (None, [_int, _int, _int, _int]),
+    "gnorm_set_tuning": (None, [_int, _int, _int, _int, _int, _int]),
     "gnorm_build_info": (ctypes.c_char_p, []),
 }
 

@@ -262,6 +262,26 @@ int gnorm_ckpt_step(const void* x, const void* g, const void* w, float eps, cons
   return enqueue_bwd(d, dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic, M, N, workspace, s);
 }
 
+int gnorm_dw_reduce(const float* partials, int64_t P, int64_t N, void* dw, int dw_fp32,
+                    void* stream) {
+  if (P < 0 || P > (int64_t(1) << 31) - 1 || N < 8 || N > GNORM_N_MAX || (N % 8) != 0)
+    return GNORM_ERR_SHAPE;
+  if (!dw) return GNORM_ERR_NULL;
+  if (!aligned(dw, 16)) return GNORM_ERR_ALIGN;
+  const size_t dw_bytes = static_cast<size_t>(N) * (dw_fp32 ? 4 : 2);
+  const cudaStream_t s = as_stream(stream);
+  if (P == 0) return cudaMemsetAsync(dw, 0, dw_bytes, s) == cudaSuccess ? GNORM_OK : GNORM_ERR_CUDA;
+  if (!partials) return GNORM_ERR_NULL;
+  if (!aligned(partials, 16)) return GNORM_ERR_ALIGN;
+  const Span in[] = {{partials, static_cast<size_t>(P) * N * 4}};
+  const Span out[] = {{dw, dw_bytes}};
+  if (any_alias(in, 1, out, 1)) return GNORM_ERR_ALIAS;
+  if (launch_dw_reduce(partials, static_cast<int>(P), static_cast<int>(N), dw, dw_fp32 ? 1 : 0,
+                       nullptr, s, use_pdl()) != cudaSuccess)
+    return GNORM_ERR_CUDA;
+  return GNORM_OK;
+}
+
 size_t gnorm_bwd_workspace_bytes_for(int64_t M, int64_t N, int deterministic, int num_sms) {
   gnorm_plan plan;
   if (check_shape(M, N) != GNORM_OK) return 0;
@@ -312,12 +332,15 @@ int gnorm_device_error(int reset) {
   return static_cast<int>(v);
 }
 
-void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl) {
+void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl,
+                      int threads_per_row, int chunks_per_thread) {
   TuningKnobs k;
   k.stage_bytes = stage_bytes > 0 ? stage_bytes : 0;
   k.max_stages = max_stages > 0 ? max_stages : 0;
   k.ctas_per_sm = ctas_per_sm > 0 ? ctas_per_sm : 0;
   k.disable_pdl = disable_pdl ? 1 : 0;
+  k.threads_per_row = threads_per_row > 0 ? threads_per_row : 0;
+  k.chunks_per_thread = chunks_per_thread > 0 ? chunks_per_thread : 0;
   set_tuning(k);
 }
 

@@ -12,8 +12,9 @@
 // Design: the same persistent, warp-specialised TMA pipeline as the forward, with three
 // tensors (dy, x, g) per stage.  Pass 1 recomputes xhat and the gate from shared memory,
 // writes dg, accumulates the row dot product sum(u xhat) and this thread's dw columns in
-// FP32 registers, and keeps u in registers; after the row reduction pass 2 re-reads x and
-// writes dx.  At the end each CTA adds its row groups' dw accumulators in a fixed order into one
+// FP32 registers (arithmetic on packed FP32 pairs), and keeps u in registers; after the row
+// reduction pass 2 re-reads x and writes dx.  The producer warp also stages the rows' rstd
+// with 4-byte asynchronous copies tracked by the same stage barrier.  At the end each CTA adds its row groups' dw accumulators in a fixed order into one
 // FP32 partial row [P, N] in the workspace.  A second launch (or, in the non-deterministic
 // mode for narrow rows, the last CTA to finish) sums the P partials in a fixed tree order
 // and writes dw once, rounded to BF16 or kept in FP32.
@@ -100,7 +101,7 @@ __global__ void __launch_bounds__(kReduceThreads)
 }
 
 template <int TPR, int CPT>
-__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
+__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(1, TPR, CPT))
     gated_rmsnorm_bwd_kernel(const BwdArgs a) {
   constexpr int kNCT = consumer_threads_for(TPR);
   constexpr int kGroups = kNCT / TPR;
@@ -116,11 +117,12 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
   const int R = a.rows_per_stage;
   const int N = a.N;
   const uint32_t tensor_bytes = static_cast<uint32_t>(R) * N * 2u;
-  const uint32_t stage_bytes = (3u * tensor_bytes + 127u) & ~127u;
+  const uint32_t stage_bytes = (3u * tensor_bytes + static_cast<uint32_t>(R) * 4u + 127u) & ~127u;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(&full[s], 1);
+      // 32 producer lanes' asynchronous rstd copies + the producer's own arrival
+      mbar_init(&full[s], 33);
       mbar_init(&empty[s], kNCT / 32);
     }
     fence_barrier_init();
@@ -133,35 +135,50 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
   const int lane = threadIdx.x & 31;
 
   if (warp == 0) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      int s = 0;
-      uint32_t phase = 0;
-      long long next = blockIdx.x;
-      while (true) {
-        const long long blk =
-            a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
-        next += gridDim.x;
-        if (!mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty)) break;
-        if (blk >= a.num_blocks) {
-          blk_id[s] = -1;
-          mbar_arrive(&full[s]);
-          break;
-        }
+    // ---------------- producer warp ----------------
+    // Lane 0 takes the next row block, waits for a free stage and issues the bulk copies of
+    // dy, x and g; all 32 lanes copy the block's rstd values with 4-byte asynchronous copies
+    // whose completion the stage's barrier also tracks.
+    int s = 0;
+    uint32_t phase = 0;
+    long long next = blockIdx.x;
+    while (true) {
+      long long blk = 0;
+      bool ok = true;
+      if (lane == 0) {
+        blk = a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
+        ok = mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty);
+      }
+      next += gridDim.x;
+      blk = __shfl_sync(0xffffffffu, blk, 0);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      __syncwarp();
+      if (!ok) break;
+      if (blk >= a.num_blocks) {
+        if (lane == 0) blk_id[s] = -1;
+        async_copies_arrive(&full[s]);
+        if (lane == 0) mbar_arrive(&full[s]);
+        break;
+      }
+      const long long r0 = blk * R;
+      const long long left = a.M - r0;
+      const int rows = static_cast<int>(left < R ? left : R);
+      uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
+      if (lane == 0) {
         blk_id[s] = blk;
-        const long long r0 = blk * R;
-        const long long left = a.M - r0;
-        const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
-        const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
-        uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
-        mbar_arrive_expect_tx(&full[s], 3u * bytes);
+        const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(N) * 2u;
+        mbar_expect_tx(&full[s], 3u * bytes);
         bulk_copy_g2s(st, a.dy + r0 * N, bytes, &full[s]);
         bulk_copy_g2s(st + tensor_bytes, a.x + r0 * N, bytes, &full[s]);
         bulk_copy_g2s(st + 2u * tensor_bytes, a.g + r0 * N, bytes, &full[s]);
-        if (++s == S) {
-          s = 0;
-          phase ^= 1u;
-        }
+      }
+      float* srs = reinterpret_cast<float*>(st + 3u * tensor_bytes);
+      for (int i = lane; i < rows; i += 32) async_copy_4(srs + i, a.rstd + r0 + i);
+      async_copies_arrive(&full[s]);
+      if (lane == 0) mbar_arrive(&full[s]);
+      if (++s == S) {
+        s = 0;
+        phase ^= 1u;
       }
     }
     return;
@@ -173,19 +190,19 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
   const int lr = ctid - group * TPR;
   const int n8 = N >> 3;
 
-  float wf[CPT][8];
-  float dwacc[CPT][8];
+  float2 wp[CPT][4];     // this thread's weights, as FP32 pairs
+  float2 dwacc[CPT][4];  // this thread's dw columns, accumulated over its rows
   bool cval[CPT];
 #pragma unroll
   for (int k = 0; k < CPT; ++k) {
     const int c = k * TPR + lr;
     cval[k] = c < n8;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      wf[k][e] = 0.f;
-      dwacc[k][e] = 0.f;
+    for (int i = 0; i < 4; ++i) {
+      wp[k][i] = splat2(0.f);
+      dwacc[k][i] = splat2(0.f);
     }
-    if (cval[k]) bf16x8_to_f32(*reinterpret_cast<const uint4*>(a.w + c * 8), wf[k]);
+    if (cval[k]) bf16x8_to_pairs(*reinterpret_cast<const uint4*>(a.w + c * 8), wp[k]);
   }
 
   int s = 0;
@@ -201,6 +218,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
     const uint8_t* sdy = stage0 + static_cast<size_t>(s) * stage_bytes;
     const uint8_t* sx = sdy + tensor_bytes;
     const uint8_t* sg = sx + tensor_bytes;
+    const float* srs = reinterpret_cast<const float*>(sg + tensor_bytes);
 
     for (int rb = 0; rb < rows; rb += kGroups) {
       const int row = rb + group;
@@ -208,39 +226,42 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
       const int srow = valid ? row : 0;
       const size_t roff = static_cast<size_t>(srow) * N * 2;
       const long long grow = r0 + row;
-      const float r = valid ? __ldg(a.rstd + grow) : 0.f;
+      const float r = srs[srow];
+      const float2 r2 = splat2(r);
 
       // pass 1: recompute xhat and the gate; dg; row dot product; dw accumulators
-      float u[CPT][8];
-      float dot = 0.f;
+      float2 u[CPT][4];
+      float2 dot2 = splat2(0.f);
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
         if (cval[k]) {
           const int c = k * TPR + lr;
           const size_t off = roff + static_cast<size_t>(c) * 16;
-          float dyf[8], xf[8], gf[8], dgf[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sdy + off), dyf);
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sx + off), xf);
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sg + off), gf);
+          float2 dyp[4], xp[4], gp[4], dgp[4];
+          bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
+          bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
+          bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sg + off), gp);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float xhat = xf[e] * r;
-            const float sgm = sigmoid_f32(gf[e]);
-            const float silu = gf[e] * sgm;
-            const float t = dyf[e] * xhat;                   // dy xhat
-            const float ue = (dyf[e] * wf[k][e]) * silu;      // dy w s
-            u[k][e] = ue;
-            dot = fmaf(ue, xhat, dot);
-            dwacc[k][e] = valid ? fmaf(t, silu, dwacc[k][e]) : dwacc[k][e];
-            dgf[e] = ((t * wf[k][e]) * sgm) * ((1.0f + gf[e]) - silu);
+          for (int i = 0; i < 4; ++i) {
+            const float2 xhat = mul2(xp[i], r2);
+            const float2 sgm = sigmoid2(gp[i]);
+            const float2 silu = mul2(gp[i], sgm);
+            const float2 t = mul2(dyp[i], xhat);                    // dy xhat
+            const float2 ue = mul2(mul2(dyp[i], wp[k][i]), silu);    // dy w s
+            u[k][i] = ue;
+            dot2 = fma2(ue, xhat, dot2);
+            if (valid) dwacc[k][i] = fma2(t, silu, dwacc[k][i]);
+            // sigmoid' (1 + g (1 - sigmoid)) written as (1 + g) - silu
+            const float2 dsilu = fma2(silu, splat2(-1.0f), add2(gp[i], splat2(1.0f)));
+            dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), dsilu);
           }
           if (valid)
-            *reinterpret_cast<uint4*>(a.dg + grow * N + c * 8) = f32x8_to_bf16(dgf);
+            *reinterpret_cast<uint4*>(a.dg + grow * N + c * 8) = pairs_to_bf16x8(dgp);
         }
       }
-      dot = row_sum<TPR>(dot, red_slots, group, lr, slot);
+      const float dot = row_sum<TPR>(dot2.x + dot2.y, red_slots, group, lr, slot);
       slot ^= 1;
-      const float rc = r * (dot * a.inv_n);
+      const float2 nrc2 = splat2(-(r * (dot * a.inv_n)));
 
       // pass 2: dx = r u - (r c) xhat, with xhat recomputed from the staged x (this keeps
       // u, w and the dw accumulators as the only per-element registers)
@@ -248,13 +269,14 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
       for (int k = 0; k < CPT; ++k) {
         if (cval[k]) {
           const int c = k * TPR + lr;
-          float xf[8], dxf[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(c) * 16),
-                        xf);
+          float2 xp[4], dxp[4];
+          bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(c) * 16),
+                          xp);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) dxf[e] = fmaf(-rc, xf[e] * r, r * u[k][e]);
+          for (int i = 0; i < 4; ++i)
+            dxp[i] = fma2(nrc2, mul2(xp[i], r2), mul2(r2, u[k][i]));
           if (valid)
-            *reinterpret_cast<uint4*>(a.dx + grow * N + c * 8) = f32x8_to_bf16(dxf);
+            *reinterpret_cast<uint4*>(a.dx + grow * N + c * 8) = pairs_to_bf16x8(dxp);
         }
       }
     }
@@ -274,8 +296,8 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
     for (int k = 0; k < CPT; ++k) {
       if (cval[k]) {
         float4* p4 = reinterpret_cast<float4*>(prow + (k * TPR + lr) * 8);
-        p4[0] = make_float4(dwacc[k][0], dwacc[k][1], dwacc[k][2], dwacc[k][3]);
-        p4[1] = make_float4(dwacc[k][4], dwacc[k][5], dwacc[k][6], dwacc[k][7]);
+        p4[0] = make_float4(dwacc[k][0].x, dwacc[k][0].y, dwacc[k][1].x, dwacc[k][1].y);
+        p4[1] = make_float4(dwacc[k][2].x, dwacc[k][2].y, dwacc[k][3].x, dwacc[k][3].y);
       }
     }
   } else {
@@ -284,8 +306,8 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
     for (int k = 0; k < CPT; ++k) {
       if (cval[k]) {
         float4* r4 = reinterpret_cast<float4*>(red + group * N + (k * TPR + lr) * 8);
-        r4[0] = make_float4(dwacc[k][0], dwacc[k][1], dwacc[k][2], dwacc[k][3]);
-        r4[1] = make_float4(dwacc[k][4], dwacc[k][5], dwacc[k][6], dwacc[k][7]);
+        r4[0] = make_float4(dwacc[k][0].x, dwacc[k][0].y, dwacc[k][1].x, dwacc[k][1].y);
+        r4[1] = make_float4(dwacc[k][2].x, dwacc[k][2].y, dwacc[k][3].x, dwacc[k][3].y);
       }
     }
     named_barrier_sync(15, kNCT);

@@ -131,11 +131,70 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float f[8]) {
   return v;
 }
 
-// Logistic function 1 / (1 + e^-t) with the fast exponential and the approximate
-// division intrinsics (one MUFU exp2 and one MUFU reciprocal).  Relative error is a few
-// FP32 ulp; for t < -88 the result is 0 (true value < 1e-38), for large t it is 1.
-__device__ __forceinline__ float sigmoid_f32(float t) {
-  return __fdividef(1.0f, 1.0f + __expf(-t));
+// Posts the bytes a stage's bulk copies will deliver, without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// 4-byte asynchronous copy global -> shared (LDGSTS), and an arrive on `bar` that fires
+// once all of this thread's earlier asynchronous copies have landed (the arrival was
+// counted in the barrier's initial count, hence .noinc).
+__device__ __forceinline__ void async_copy_4(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(smem_dst)),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void async_copies_arrive(uint64_t* bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+// ---- packed FP32 pairs (sm_100 FFMA2 / FMUL2 / FADD2: two lanes of FP32 per instruction)
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 splat2(float v) { return make_float2(v, v); }
+
+// Eight BF16 values in a 16-byte word -> four FP32 pairs (element 2i in .x, 2i+1 in .y).
+__device__ __forceinline__ void bf16x8_to_pairs(const uint4 v, float2 p[4]) {
+  p[0] = make_float2(__uint_as_float(v.x << 16), __uint_as_float(v.x & 0xffff0000u));
+  p[1] = make_float2(__uint_as_float(v.y << 16), __uint_as_float(v.y & 0xffff0000u));
+  p[2] = make_float2(__uint_as_float(v.z << 16), __uint_as_float(v.z & 0xffff0000u));
+  p[3] = make_float2(__uint_as_float(v.w << 16), __uint_as_float(v.w & 0xffff0000u));
+}
+
+__device__ __forceinline__ uint4 pairs_to_bf16x8(const float2 p[4]) {
+  uint4 v;
+  v.x = pack_bf16x2(p[0].x, p[0].y);
+  v.y = pack_bf16x2(p[1].x, p[1].y);
+  v.z = pack_bf16x2(p[2].x, p[2].y);
+  v.w = pack_bf16x2(p[3].x, p[3].y);
+  return v;
+}
+
+__device__ __forceinline__ float ex2_approx(float v) {
+  float r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ float rcp_approx(float v) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(v));
+  return r;
+}
+
+// Logistic function of a pair, sigma(t) = 1 / (1 + 2^(-t log2(e))): the MUFU exp2 and
+// reciprocal approximations (each a few FP32 ulp) with the scaling and the +1 as packed
+// pair instructions.  For t < -88 the sum overflows to +inf and sigma = 0 (true value
+// below 2^-126); for large t, sigma = 1.
+constexpr float kLog2e = 1.4426950408889634f;
+__device__ __forceinline__ float2 sigmoid2(float2 t) {
+  const float2 z = mul2(t, splat2(-kLog2e));
+  float2 d = make_float2(ex2_approx(z.x), ex2_approx(z.y));
+  d = add2(d, splat2(1.0f));
+  return make_float2(rcp_approx(d.x), rcp_approx(d.y));
 }
 
 // Sum over the `TPR` consecutive threads that share a row.  TPR <= 32: butterfly

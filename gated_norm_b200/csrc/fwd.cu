@@ -23,7 +23,11 @@ cudaError_t launch_fwd(const gnorm_plan& p, const FwdArgs& a, cudaStream_t strea
     case 32 * 8 + 1: return launch_fwd_geometry<32, 1>(p, a, stream, pdl);
     case 32 * 8 + 2: return launch_fwd_geometry<32, 2>(p, a, stream, pdl);
     case 32 * 8 + 4: return launch_fwd_geometry<32, 4>(p, a, stream, pdl);
+    case 64 * 8 + 2: return launch_fwd_geometry<64, 2>(p, a, stream, pdl);
     case 64 * 8 + 4: return launch_fwd_geometry<64, 4>(p, a, stream, pdl);
+    case 128 * 8 + 2: return launch_fwd_geometry<128, 2>(p, a, stream, pdl);
+    case 256 * 8 + 2: return launch_fwd_geometry<256, 2>(p, a, stream, pdl);
+    case 64 * 8 + 8: return launch_fwd_geometry<64, 8>(p, a, stream, pdl);
     case 128 * 8 + 4: return launch_fwd_geometry<128, 4>(p, a, stream, pdl);
     case 256 * 8 + 4: return launch_fwd_geometry<256, 4>(p, a, stream, pdl);
     case 512 * 8 + 4: return launch_fwd_geometry<512, 4>(p, a, stream, pdl);

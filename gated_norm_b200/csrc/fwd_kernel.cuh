@@ -23,7 +23,7 @@ namespace gnorm {
 
 
 template <int TPR, int CPT>
-__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
+__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(0, TPR, CPT))
     gated_rmsnorm_fwd_kernel(const FwdArgs a) {
   constexpr int kNCT = consumer_threads_for(TPR);
   constexpr int kGroups = kNCT / TPR;
@@ -91,19 +91,15 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
   const int lr = ctid - group * TPR;    // thread index inside the row
   const int n8 = N >> 3;                // 16-byte chunks per row
 
-  float wf[CPT][8];
+  float2 wp[CPT][4];  // this thread's weights, as FP32 pairs
   bool cval[CPT];
 #pragma unroll
   for (int k = 0; k < CPT; ++k) {
     const int c = k * TPR + lr;
     cval[k] = c < n8;
-    if (cval[k]) {
-      const uint4 wv = *reinterpret_cast<const uint4*>(a.w + c * 8);
-      bf16x8_to_f32(wv, wf[k]);
-    } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) wf[k][e] = 0.f;
-    }
+    for (int i = 0; i < 4; ++i) wp[k][i] = splat2(0.f);
+    if (cval[k]) bf16x8_to_pairs(*reinterpret_cast<const uint4*>(a.w + c * 8), wp[k]);
   }
 
   int s = 0;
@@ -125,41 +121,42 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, 1)
       const int srow = valid ? row : 0;  // keep shared-memory reads inside the stage
       const size_t roff = static_cast<size_t>(srow) * N * 2;
 
-      // pass 1: sum of squares of the row
+      // pass 1: sum of squares of the row (two interleaved FP32 partial sums per thread)
       uint4 xv[CPT];
-      float ss = 0.f;
+      float2 ss2 = splat2(0.f);
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
         if (cval[k]) {
           xv[k] = *reinterpret_cast<const uint4*>(sx + roff + (k * TPR + lr) * 16);
-          float f[8];
-          bf16x8_to_f32(xv[k], f);
+          float2 xp[4];
+          bf16x8_to_pairs(xv[k], xp);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) ss = fmaf(f[e], f[e], ss);
+          for (int i = 0; i < 4; ++i) ss2 = fma2(xp[i], xp[i], ss2);
         }
       }
-      ss = row_sum<TPR>(ss, red_slots, group, lr, slot);
+      const float ss = row_sum<TPR>(ss2.x + ss2.y, red_slots, group, lr, slot);
       slot ^= 1;
       const float r = rsqrtf(fmaf(ss, a.inv_n, a.eps));
       const long long grow = r0 + row;
       if (valid && lr == 0) a.rstd[grow] = r;
 
-      // pass 2: y = xhat * w * g * sigmoid(g)
+      // pass 2: y = ((x r) w) (g sigmoid(g))
+      const float2 r2 = splat2(r);
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
         if (cval[k]) {
           const int c = k * TPR + lr;
           const uint4 gv = *reinterpret_cast<const uint4*>(sg + roff + c * 16);
-          float xf[8], gf[8], yf[8];
-          bf16x8_to_f32(xv[k], xf);
-          bf16x8_to_f32(gv, gf);
+          float2 xp[4], gp[4], yp[4];
+          bf16x8_to_pairs(xv[k], xp);
+          bf16x8_to_pairs(gv, gp);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float silu = gf[e] * sigmoid_f32(gf[e]);
-            yf[e] = ((xf[e] * r) * wf[k][e]) * silu;
+          for (int i = 0; i < 4; ++i) {
+            const float2 silu = mul2(gp[i], sigmoid2(gp[i]));
+            yp[i] = mul2(mul2(mul2(xp[i], r2), wp[k][i]), silu);
           }
           if (valid)
-            *reinterpret_cast<uint4*>(a.y + grow * N + c * 8) = f32x8_to_bf16(yf);
+            *reinterpret_cast<uint4*>(a.y + grow * N + c * 8) = pairs_to_bf16x8(yp);
         }
       }
     }

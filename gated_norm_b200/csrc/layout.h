@@ -21,4 +21,13 @@ GNORM_HD constexpr int consumer_threads_for(int threads_per_row) {
   return threads_per_row > 256 ? threads_per_row : 256;
 }
 
+// Resident CTAs per SM a kernel is compiled for (its __launch_bounds__ minimum), which caps
+// its registers: 3 CTAs of 288 threads leave 75 registers per thread, 2 leave 113.  The
+// dispatch rule never plans more CTAs per SM than this.
+GNORM_HD constexpr int max_ctas_per_sm(int kind, int threads_per_row, int chunks_per_thread) {
+  return threads_per_row > 256 ? 1
+         : kind == 0            ? (chunks_per_thread == 1 ? 3 : (chunks_per_thread <= 4 ? 2 : 1))
+                                : (chunks_per_thread == 1 ? 2 : 1);
+}
+
 }  // namespace gnorm

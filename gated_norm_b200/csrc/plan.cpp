@@ -3,12 +3,14 @@
 // flashinfer PR #8701 ("perf(cake_rmsnorm_silu_gate_train): L2-prefetching extra-long
 // forward on SM107", PR description and commit message) routes its forward by architecture
 // and by rows per SM (M / #SMs) into "long" and "extra-long" tiers with per-architecture
-// thresholds.  This rule is this library's own for B200: it picks a row geometry from N,
-// then sizes the pipeline stage from the bytes one row brings in, and splits the rows
-// evenly over one persistent CTA per SM.  The tiers are:
-//   rows per SM <= the stage's target rows : one block per CTA (latency tier, small M);
-//   otherwise                              : k blocks per CTA, block size chosen so all
-//                                            CTAs get the same number of rows (streaming).
+// thresholds.  This rule is this library's own for B200: it picks a row geometry from N
+// (about two 16-byte chunks per thread), sets CTAs per SM and the stage size by a rows-per-SM
+// tier, and splits the rows evenly over the persistent CTAs:
+//   forward with < 512 KB of staged rows per SM : 3 CTAs per SM, ~16 KB stages (latency tier);
+//   other forwards                              : 2 CTAs per SM, ~48 KB stages;
+//   backward                                    : 1 CTA per SM, ~48 KB (>= 3-row) stages;
+// and within a tier: if the rows per CTA fit in one stage, one block per CTA; otherwise k
+// equal blocks per CTA, block size chosen so all CTAs get the same number of rows.
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -24,16 +26,29 @@ static TuningKnobs g_knobs;  // all zero: built-in values
 void set_tuning(const TuningKnobs& k) { g_knobs = k; }
 TuningKnobs get_tuning() { return g_knobs; }
 
+bool geometry_compiled(int kind, int tpr, int cpt) {
+  static const int kBoth[][2] = {{4, 1},   {8, 1},   {16, 1},  {32, 1},  {32, 2},
+                                 {32, 4},  {64, 2},  {64, 4},  {128, 2}, {128, 4},
+                                 {256, 2}, {256, 4}, {512, 4}};
+  static const int kFwdOnly[][2] = {{64, 8}};
+  for (const auto& g : kBoth)
+    if (g[0] == tpr && g[1] == cpt) return true;
+  if (kind == 0)
+    for (const auto& g : kFwdOnly)
+      if (g[0] == tpr && g[1] == cpt) return true;
+  return false;
+}
+
 RowGeometry geometry_for(int64_t N) {
-  const int64_t n8 = N / 8;
+  const int64_t n8 = N / 8;  // 16-byte chunks per row
   if (n8 <= 4) return {4, 1};
   if (n8 <= 8) return {8, 1};
   if (n8 <= 16) return {16, 1};
   if (n8 <= 32) return {32, 1};
   if (n8 <= 64) return {32, 2};
-  if (n8 <= 128) return {32, 4};
-  if (n8 <= 256) return {64, 4};
-  if (n8 <= 512) return {128, 4};
+  if (n8 <= 128) return {64, 2};
+  if (n8 <= 256) return {128, 2};
+  if (n8 <= 512) return {256, 2};
   if (n8 <= 1024) return {256, 4};
   return {512, 4};
 }
@@ -49,14 +64,28 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   if (num_sms <= 0) return GNORM_ERR_ARG;
   if (smem_per_block <= 0) smem_per_block = kB200SmemPerBlock;
 
-  const RowGeometry geo = geometry_for(N);
+  RowGeometry geo = geometry_for(N);
+  if (g_knobs.threads_per_row > 0 && g_knobs.chunks_per_thread > 0) {
+    geo = {g_knobs.threads_per_row, g_knobs.chunks_per_thread};
+    if (!geometry_compiled(kind, geo.threads_per_row, geo.chunks_per_thread) ||
+        static_cast<int64_t>(geo.threads_per_row) * geo.chunks_per_thread * 8 < N)
+      return GNORM_ERR_UNSUPPORTED;
+  }
   const int nct = consumer_threads_for(geo.threads_per_row);
   const int groups = nct / geo.threads_per_row;
   const int tensors = kind == 0 ? 2 : 3;
   const int64_t row_bytes = static_cast<int64_t>(tensors) * N * 2;
 
-  const int ctas_per_sm = g_knobs.ctas_per_sm > 0 ? g_knobs.ctas_per_sm : 1;
-  const int64_t stage_target = g_knobs.stage_bytes > 0 ? g_knobs.stage_bytes : kStageTargetBytes;
+  // Rows-per-SM tiers (bytes of staged rows per SM decide, so wide and narrow rows compare).
+  const int64_t rows_per_sm = (M + num_sms - 1) / num_sms;
+  const bool latency_tier = kind == 0 && rows_per_sm * row_bytes < kFwdLatencyTierBytes;
+  const int fit = max_ctas_per_sm(kind, geo.threads_per_row, geo.chunks_per_thread);
+  const int default_ctas = kind == 1 ? 1 : (latency_tier ? 3 : 2);
+  int64_t default_stage = kind == 1 ? std::max<int64_t>(kBwdStageBytes, kBwdMinStageRows * (row_bytes + 4))
+                                    : (latency_tier ? kFwdLatencyStageBytes : kFwdStageBytes);
+  const int ctas_per_sm =
+      std::min(fit, g_knobs.ctas_per_sm > 0 ? g_knobs.ctas_per_sm : default_ctas);
+  const int64_t stage_target = g_knobs.stage_bytes > 0 ? g_knobs.stage_bytes : default_stage;
   const int max_stages =
       std::min(kMaxStages, g_knobs.max_stages > 0 ? g_knobs.max_stages : kMaxStages);
 
@@ -67,9 +96,10 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   const int64_t budget = smem_cta - kHeaderBytes;
 
   // Rows per stage: about `stage_target` bytes, at least one row per row group.
-  int64_t target_rows = std::max<int64_t>(groups, stage_target / row_bytes);
-  while (target_rows > 1 && 2 * target_rows * row_bytes > budget) --target_rows;
-  if (2 * row_bytes > budget) return GNORM_ERR_UNSUPPORTED;  // two stages of one row
+  const int64_t row_stage_bytes = row_bytes + (kind == 1 ? 4 : 0);
+  int64_t target_rows = std::max<int64_t>(groups, stage_target / row_stage_bytes);
+  while (target_rows > 1 && 2 * (target_rows * row_stage_bytes + 127) > budget) --target_rows;
+  if (2 * (row_stage_bytes + 127) > budget) return GNORM_ERR_UNSUPPORTED;  // two stages of one row
 
   const int64_t grid_max = static_cast<int64_t>(num_sms) * ctas_per_sm;
   int64_t R, blocks, grid;
@@ -89,7 +119,9 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
     grid = std::min(blocks, grid_max);
   }
 
-  const int64_t stage_bytes = (static_cast<int64_t>(tensors) * R * N * 2 + 127) / 128 * 128;
+  // A stage holds R rows of each tensor; the backward's also holds their R FP32 rstd values.
+  const int64_t stage_raw = static_cast<int64_t>(tensors) * R * N * 2 + (kind == 1 ? R * 4 : 0);
+  const int64_t stage_bytes = (stage_raw + 127) / 128 * 128;
   int64_t stages = std::min<int64_t>(max_stages, budget / stage_bytes);
   if (stages < 2) return GNORM_ERR_UNSUPPORTED;
 

@@ -20,6 +20,7 @@ __all__ = [
     "gnorm_bwd",
     "gnorm_ckpt_step",
     "gnorm_bwd_noalloc",
+    "gnorm_dw_reduce",
     "gnorm_bwd_workspace_bytes",
     "gnorm_bwd_workspace_bytes_for",
     "gnorm_status_string",
@@ -70,9 +71,10 @@ def gnorm_device_error(reset: bool = False) -> int:
 
 
 def gnorm_set_tuning(stage_bytes: int = 0, max_stages: int = 0, ctas_per_sm: int = 0,
-                     disable_pdl: bool = False) -> None:
+                     disable_pdl: bool = False, threads_per_row: int = 0,
+                     chunks_per_thread: int = 0) -> None:
     lib.gnorm_set_tuning(int(stage_bytes), int(max_stages), int(ctas_per_sm),
-                         int(bool(disable_pdl)))
+                         int(bool(disable_pdl)), int(threads_per_row), int(chunks_per_thread))
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -201,6 +203,23 @@ def gnorm_bwd(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: bool = F
                            ws.numel() * ws.element_size(), _stream(stream, x.device))
     _check(st, "gnorm_bwd")
     return dx, dg, dw
+
+
+def gnorm_dw_reduce(partials, *, dw=None, dw_fp32: bool = True, stream=None):
+    """Fixed-order sum of FP32 partial rows [P, N] into dw [N] (BF16 or FP32)."""
+    if partials.dtype != torch.float32 or partials.dim() != 2 or not partials.is_contiguous():
+        raise ValueError("partials must be a contiguous FP32 [P, N] CUDA tensor")
+    P, N = partials.shape
+    dw_dtype = torch.float32 if dw_fp32 else torch.bfloat16
+    if dw is None:
+        dw = torch.empty(N, dtype=dw_dtype, device=partials.device)
+    else:
+        _vec(dw, N, (dw_dtype,), "dw", partials.device)
+    with torch.cuda.device(partials.device):
+        st = lib.gnorm_dw_reduce(_ptr(partials), P, N, _ptr(dw), int(bool(dw_fp32)),
+                                 _stream(stream, partials.device))
+    _check(st, "gnorm_dw_reduce")
+    return dw
 
 
 def gnorm_bwd_noalloc(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: bool = False,

@@ -132,6 +132,18 @@ GNORM_API int gnorm_ckpt_step(const void* x, const void* g, const void* w, float
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Fixed-order sum of P rows of FP32 partials [P, N] (device memory, row-major) into dw[N]
+ * (BF16 if dw_fp32 == 0, else FP32), with the same kernel and summation order as the
+ * backward's deterministic second pass (the fixed-order FP32 partial reduction of flashinfer
+ * PR #8878's commit message).  Data-parallel training uses it to combine per-rank FP32 dw
+ * gathered in rank order: every rank then holds bitwise the same dw, independent of the
+ * collective's own reduction order.  P == 0 writes dw = 0.  partials and dw 16-byte aligned,
+ * not overlapping; N a multiple of 8 up to GNORM_N_MAX.
+ */
+GNORM_API int gnorm_dw_reduce(const float* partials, int64_t P, int64_t N, void* dw, int dw_fp32,
+                              void* stream);
+
+/*
  * Workspace bytes gnorm_bwd / gnorm_ckpt_step need on the CURRENT device (reads its SM count).
  * Returns 0 if the arguments are invalid or no device is present.
  */
@@ -183,11 +195,14 @@ GNORM_API int gnorm_device_error(int reset);
 
 /*
  * Process-wide tuning knobs for experiments (0 keeps the built-in value): target bytes per
- * pipeline stage, maximum pipeline depth, resident CTAs per SM, and 1 to launch without
- * programmatic dependent launch.  Affects plans made after the call, including
+ * pipeline stage, maximum pipeline depth, resident CTAs per SM, 1 to launch without
+ * programmatic dependent launch, and a forced row geometry (threads per row and 16-byte
+ * chunks per thread; both must name a compiled geometry that covers N, else plans fail
+ * with GNORM_ERR_UNSUPPORTED).  Affects plans made after the call, including
  * gnorm_plan_query and gnorm_bwd_workspace_bytes.  Not thread-safe with concurrent calls.
  */
-GNORM_API void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl);
+GNORM_API void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl,
+                                int threads_per_row, int chunks_per_thread);
 
 /* Build description: compiler version, target architecture (static storage). */
 GNORM_API const char* gnorm_build_info(void);

@@ -89,7 +89,7 @@ def test_plan_invariants(sms, kind):
                 assert p["consumer_threads"] % p["threads_per_row"] == 0
                 assert p["consumer_threads"] + 32 <= 1024
                 tensors = 2 if kind == 0 else 3
-                stage = -(-tensors * R * N * 2 // 128) * 128
+                stage = -(-(tensors * R * N * 2 + (4 * R if kind == 1 else 0)) // 128) * 128
                 assert p["smem_bytes"] >= 1024 + p["stages"] * stage
                 assert p["smem_bytes"] <= 232448
                 # static round-robin: no CTA gets more than one block above the mean
@@ -111,21 +111,58 @@ def test_plan_is_a_pure_function():
 
 
 def test_tier_edge_rows_per_sm():
-    """Latency tier (one block per CTA) up to the stage's target rows per SM, then the
-    streaming tier (several equal blocks per CTA) -- tested on both sides of the edge."""
+    """The rows-per-SM tiers, each tested on both sides of its edge.
+
+    Forward: under 512 KB of staged rows (x and g) per SM the latency tier runs 3 CTAs
+    per SM with small stages, from there on the streaming tier runs 2.  Within a tier,
+    one block per CTA while the CTA's rows fit one stage, then equal multi-block shares."""
     for sms in SM_COUNTS:
-        edge = None
-        for rows_per_sm in range(1, 200):
-            p = gn.gnorm_plan_query(0, rows_per_sm * sms, 128, True, sms)
-            if p["num_blocks"] > p["grid"]:
-                edge = rows_per_sm
-                break
-        assert edge is not None
-        below = gn.gnorm_plan_query(0, (edge - 1) * sms, 128, True, sms)
-        above = gn.gnorm_plan_query(0, edge * sms, 128, True, sms)
-        assert below["num_blocks"] == below["grid"] == sms
-        assert above["num_blocks"] > above["grid"]
-        assert above["rows_per_stage"] * 2 >= below["rows_per_stage"]
+        N = 128
+        rows_edge = 512 * 1024 // (4 * N)  # rows per SM where the staged bytes reach 512 KB
+        lat = gn.gnorm_plan_query(0, (rows_edge - 1) * sms, N, True, sms)
+        stream = gn.gnorm_plan_query(0, rows_edge * sms, N, True, sms)
+        assert lat["ctas_per_sm"] == 3 and stream["ctas_per_sm"] == 2
+        assert lat["rows_per_stage"] * 4 * N <= 16384 < stream["rows_per_stage"] * 4 * N
+        # the wide-row forward uses the same byte rule; its registers cap it at 2 CTAs per SM
+        wide_lat = gn.gnorm_plan_query(0, 8 * sms, 4096, True, sms)
+        wide_stream = gn.gnorm_plan_query(0, 64 * sms, 4096, True, sms)
+        assert wide_lat["ctas_per_sm"] == wide_stream["ctas_per_sm"] == 2
+        assert wide_lat["rows_per_stage"] == 1 and wide_stream["rows_per_stage"] == 3
+        for kind in (0, 1):
+            big = gn.gnorm_plan_query(kind, 1 << 12, N, True, sms)
+            ctas = sms * big["ctas_per_sm"]
+            edge = None
+            for rows_per_cta in range(1, 400):
+                p = gn.gnorm_plan_query(kind, rows_per_cta * ctas, N, True, sms)
+                if p["ctas_per_sm"] != big["ctas_per_sm"]:
+                    break
+                if p["num_blocks"] > p["grid"]:
+                    edge = rows_per_cta
+                    break
+            if edge is None:
+                continue
+            below = gn.gnorm_plan_query(kind, (edge - 1) * ctas, N, True, sms)
+            above = gn.gnorm_plan_query(kind, edge * ctas, N, True, sms)
+            assert below["num_blocks"] == below["grid"] == ctas
+            assert below["rows_per_stage"] == edge - 1
+            assert above["num_blocks"] > above["grid"]
+
+
+def test_ctas_per_sm_never_exceeds_the_compiled_residency():
+    for kind in (0, 1):
+        for N in NS:
+            for M in MS:
+                for knob in (0, 2, 3, 4):
+                    try:
+                        gn.gnorm_set_tuning(ctas_per_sm=knob)
+                        p = gn.gnorm_plan_query(kind, M, N, True, 148)
+                    finally:
+                        gn.gnorm_set_tuning()
+                    tpr, cpt = p["threads_per_row"], p["chunks_per_thread"]
+                    fit = 1 if tpr > 256 else (
+                        (3 if cpt == 1 else 2 if cpt <= 4 else 1) if kind == 0 else
+                        (2 if cpt == 1 else 1))
+                    assert p["ctas_per_sm"] <= fit
 
 
 def test_plan_errors():
@@ -158,3 +195,21 @@ def test_tuning_knobs_change_plans_and_reset():
     finally:
         gn.gnorm_set_tuning()
     assert gn.gnorm_plan_query(0, 1 << 20, 128, True, 148) == base
+
+
+def test_forced_geometry_knob():
+    try:
+        gn.gnorm_set_tuning(threads_per_row=256, chunks_per_thread=2)
+        p = gn.gnorm_plan_query(0, 4096, 4096, True, 148)
+        assert (p["threads_per_row"], p["chunks_per_thread"]) == (256, 2)
+        with pytest.raises(gn.GnormError):  # 256 x 2 x 8 < 8192 columns
+            gn.gnorm_plan_query(0, 4096, 8192, True, 148)
+        gn.gnorm_set_tuning(threads_per_row=64, chunks_per_thread=8)
+        assert gn.gnorm_plan_query(0, 64, 4096, True, 148)["threads_per_row"] == 64
+        with pytest.raises(gn.GnormError):  # forward-only geometry
+            gn.gnorm_plan_query(1, 64, 4096, True, 148)
+        gn.gnorm_set_tuning(threads_per_row=48, chunks_per_thread=3)
+        with pytest.raises(gn.GnormError):  # not compiled
+            gn.gnorm_plan_query(0, 64, 128, True, 148)
+    finally:
+        gn.gnorm_set_tuning()
