@@ -40,11 +40,19 @@ class GnormPlan(ctypes.Structure):
         ("dynamic_schedule", ctypes.c_int),
         ("fused_reduce", ctypes.c_int),
         ("partials", ctypes.c_int),
-        ("reserved", ctypes.c_int),
+        ("l2_prefetch", ctypes.c_int),
     ]
 
     def as_dict(self) -> dict:
-        return {name: getattr(self, name) for name, _ in self._fields_ if name != "reserved"}
+        return {name: getattr(self, name) for name, _ in self._fields_}
+
+
+class GnormTuning(ctypes.Structure):
+    """Mirror of ``gnorm_tuning`` in include/gnorm.h."""
+
+    _fields_ = [(name, ctypes.c_int) for name in (
+        "stage_bytes", "max_stages", "ctas_per_sm", "disable_pdl", "threads_per_row",
+        "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch")]
 
 
 _vp = ctypes.c_void_p
@@ -68,7 +76,7 @@ SIGNATURES = {
     "gnorm_status_string": (ctypes.c_char_p, [_int]),
     "gnorm_plan_query": (_int, [_int, _i64, _i64, _int, _int, _int, ctypes.POINTER(GnormPlan)]),
     "gnorm_device_error": (_int, [_int]),
-    "gnorm_set_tuning": (None, [_int, _int, _int, _int, _int, _int]),
+    "gnorm_set_tuning": (None, [ctypes.POINTER(GnormTuning)]),
     "gnorm_build_info": (ctypes.c_char_p, []),
 }
 

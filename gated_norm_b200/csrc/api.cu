@@ -93,8 +93,11 @@ bool use_pdl() { return get_tuning().disable_pdl == 0; }
 
 cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
 
+// `prefetch`: the previous kernel on the stream is known to write none of this call's
+// inputs, so the kernel may start copying them before that kernel has finished.
 int enqueue_fwd(const DeviceInfo& d, const void* x, const void* g, const void* w, float eps,
-                void* y, float* rstd, int64_t M, int64_t N, cudaStream_t stream) {
+                void* y, float* rstd, int64_t M, int64_t N, cudaStream_t stream,
+                bool prefetch = false) {
   gnorm_plan plan;
   int st = make_plan(0, M, N, 1, d.num_sms, d.smem_optin, &plan);
   if (st != GNORM_OK) return st;
@@ -111,6 +114,8 @@ int enqueue_fwd(const DeviceInfo& d, const void* x, const void* g, const void* w
   a.rows_per_stage = plan.rows_per_stage;
   a.stages = plan.stages;
   a.num_blocks = plan.num_blocks;
+  a.prefetch = prefetch ? 1 : 0;
+  a.l2_prefetch = plan.l2_prefetch;
   a.err = d.err_word;
   if (launch_fwd(plan, a, stream, use_pdl()) != cudaSuccess) return GNORM_ERR_CUDA;
   return GNORM_OK;
@@ -118,7 +123,8 @@ int enqueue_fwd(const DeviceInfo& d, const void* x, const void* g, const void* w
 
 int enqueue_bwd(const DeviceInfo& d, const void* dy, const void* x, const void* g,
                 const void* w, const float* rstd, void* dx, void* dg, void* dw, int dw_fp32,
-                int deterministic, int64_t M, int64_t N, void* ws, cudaStream_t stream) {
+                int deterministic, int64_t M, int64_t N, void* ws, cudaStream_t stream,
+                bool prefetch = false) {
   gnorm_plan plan;
   int st = make_plan(1, M, N, deterministic, d.num_sms, d.smem_optin, &plan);
   if (st != GNORM_OK) return st;
@@ -144,6 +150,8 @@ int enqueue_bwd(const DeviceInfo& d, const void* dy, const void* x, const void* 
   a.dynamic_schedule = plan.dynamic_schedule;
   a.fused_reduce = plan.fused_reduce;
   a.dw_fp32 = dw_fp32 ? 1 : 0;
+  a.prefetch = prefetch ? 1 : 0;
+  a.l2_prefetch = plan.l2_prefetch;
   a.err = d.err_word;
   const bool pdl = use_pdl();
   if (launch_bwd(plan, a, stream, pdl) != cudaSuccess) return GNORM_ERR_CUDA;
@@ -255,11 +263,17 @@ int gnorm_ckpt_step(const void* x, const void* g, const void* w, float eps, cons
   st = check_workspace(d, M, N, deterministic, workspace, workspace_bytes);
   if (st != GNORM_OK) return st;
   const cudaStream_t s = as_stream(stream);
+  // The second forward (the recompute) follows the first, which writes only y and rstd;
+  // the backward follows it and reads rstd only after it ends.  Neither predecessor writes
+  // x, g or dy (outputs may not overlap inputs), so those copies may start early.
+  const int cp = get_tuning().chain_prefetch;
+  const bool chain = cp == 1 ? true : (cp == 2 ? false : kDefaultChainPrefetch != 0);
   st = enqueue_fwd(d, x, g, w, eps, y, rstd, M, N, s);
   if (st != GNORM_OK) return st;
-  st = enqueue_fwd(d, x, g, w, eps, y, rstd, M, N, s);  // recompute, as a checkpointed step does
+  st = enqueue_fwd(d, x, g, w, eps, y, rstd, M, N, s, chain);
   if (st != GNORM_OK) return st;
-  return enqueue_bwd(d, dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic, M, N, workspace, s);
+  return enqueue_bwd(d, dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic, M, N, workspace, s,
+                     chain);
 }
 
 int gnorm_dw_reduce(const float* partials, int64_t P, int64_t N, void* dw, int dw_fp32,
@@ -332,15 +346,22 @@ int gnorm_device_error(int reset) {
   return static_cast<int>(v);
 }
 
-void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl,
-                      int threads_per_row, int chunks_per_thread) {
-  TuningKnobs k;
-  k.stage_bytes = stage_bytes > 0 ? stage_bytes : 0;
-  k.max_stages = max_stages > 0 ? max_stages : 0;
-  k.ctas_per_sm = ctas_per_sm > 0 ? ctas_per_sm : 0;
-  k.disable_pdl = disable_pdl ? 1 : 0;
-  k.threads_per_row = threads_per_row > 0 ? threads_per_row : 0;
-  k.chunks_per_thread = chunks_per_thread > 0 ? chunks_per_thread : 0;
+void gnorm_set_tuning(const gnorm_tuning* tuning) {
+  TuningKnobs k = {};
+  if (tuning != nullptr) {
+    k = *tuning;
+    auto clamp0 = [](int v) { return v > 0 ? v : 0; };
+    auto tri = [](int v) { return (v == 1 || v == 2) ? v : 0; };
+    k.stage_bytes = clamp0(k.stage_bytes);
+    k.max_stages = clamp0(k.max_stages);
+    k.ctas_per_sm = clamp0(k.ctas_per_sm);
+    k.disable_pdl = k.disable_pdl ? 1 : 0;
+    k.threads_per_row = clamp0(k.threads_per_row);
+    k.chunks_per_thread = clamp0(k.chunks_per_thread);
+    k.l2_prefetch = tri(k.l2_prefetch);
+    k.tail_reduce = tri(k.tail_reduce);
+    k.chain_prefetch = tri(k.chain_prefetch);
+  }
   set_tuning(k);
 }
 

@@ -18,6 +18,8 @@ struct FwdArgs {
   int rows_per_stage;
   int stages;
   long long num_blocks;
+  int prefetch = 0;  // 1: the first stages' inputs may be copied before the previous grid ends
+  int l2_prefetch = 0;  // 1: also warm L2 with the block the CTA loads after the ring's
   unsigned* err;
 };
 
@@ -42,6 +44,8 @@ struct BwdArgs {
   int dynamic_schedule;
   int fused_reduce;
   int dw_fp32;
+  int prefetch = 0;  // 1: the first stages' dy, x, g may be copied before the previous grid ends
+  int l2_prefetch = 0;  // 1: also warm L2 with the block the CTA loads after the ring's
   unsigned* err;
 };
 

@@ -15,9 +15,10 @@
 // FP32 registers (arithmetic on packed FP32 pairs), and keeps u in registers; after the row
 // reduction pass 2 re-reads x and writes dx.  The producer warp also stages the rows' rstd
 // with 4-byte asynchronous copies tracked by the same stage barrier.  At the end each CTA adds its row groups' dw accumulators in a fixed order into one
-// FP32 partial row [P, N] in the workspace.  A second launch (or, in the non-deterministic
-// mode for narrow rows, the last CTA to finish) sums the P partials in a fixed tree order
-// and writes dw once, rounded to BF16 or kept in FP32.
+// FP32 partial row [P, N] in the workspace.  A second pass sums the P partials in a fixed
+// tree order and writes dw once, rounded to BF16 or kept in FP32: by default a second launch
+// whose CTAs share the columns; optionally (small partials) the backward's last CTA to
+// finish, found with an integer ticket, never a wait.
 #pragma once
 
 #include "args.h"
@@ -49,13 +50,27 @@ __device__ __forceinline__ void reduce_partials(const float* __restrict__ partia
     const bool valid = j4 < n4;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (valid) {
+      // Rows bl, bl + BL, ... in increasing order.  Loads are issued kBatch at a time
+      // before the (sequential, fixed-order) adds, so a thread waits for one memory round
+      // trip per batch instead of one per row.
+      constexpr int kBatch = 8;
       const float4* p4 = reinterpret_cast<const float4*>(partial) + j4;
-      for (int b = bl; b < P; b += BL) {
-        const float4 v = __ldcg(p4 + static_cast<size_t>(b) * n4);
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+      for (int b0 = bl; b0 < P; b0 += kBatch * BL) {
+        float4 v[kBatch];
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          const int b = b0 + i * BL;
+          v[i] = b < P ? __ldcg(p4 + static_cast<size_t>(b) * n4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int i = 0; i < kBatch; ++i) {
+          if (b0 + i * BL < P) {
+            acc.x += v[i].x;
+            acc.y += v[i].y;
+            acc.z += v[i].z;
+            acc.w += v[i].w;
+          }
+        }
       }
     }
     scratch[tid] = acc;
@@ -87,8 +102,9 @@ __device__ __forceinline__ void reduce_partials(const float* __restrict__ partia
   }
 }
 
-// Second pass of the deterministic dw: one CTA per 128 columns.  Also clears the
-// dynamic-schedule counter of the workspace (the backward grid has finished by now).
+// Second pass over the dw partials (both modes): one CTA per 128 columns.
+// Also clears the dynamic-schedule counter of the workspace (the backward grid has
+// finished by now).
 __global__ void __launch_bounds__(kReduceThreads)
     dw_reduce_kernel(const float* __restrict__ partial, int P, int N, void* dw, int dw_fp32,
                      unsigned long long* work_counter) {
@@ -128,11 +144,41 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
     fence_barrier_init();
   }
   __syncthreads();
-  grid_dependency_wait();
-  allow_dependent_launch();
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+
+  // Bulk copies of stage s's block `blk` (dy, x, g), counted on the stage's full barrier.
+  auto issue_copies = [&](int s, long long blk) {
+    const long long r0 = blk * R;
+    const long long left = a.M - r0;
+    const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
+    const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+    uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
+    mbar_expect_tx(&full[s], 3u * bytes);
+    bulk_copy_g2s(st, a.dy + r0 * N, bytes, &full[s]);
+    bulk_copy_g2s(st + tensor_bytes, a.x + r0 * N, bytes, &full[s]);
+    bulk_copy_g2s(st + 2u * tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+  };
+
+  // When the host knows the previous kernel on the stream writes none of dy, x, g (the
+  // forward of a checkpointed step), the first stages' copies of those start before it has
+  // finished.  rstd, which that forward writes, is copied only after the wait below.
+  int prefetched = 0;
+  long long pre_blk[kMaxStages];
+  if (a.prefetch && warp == 0 && lane == 0) {
+    long long next = blockIdx.x;
+    while (prefetched < S) {
+      const long long blk =
+          a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
+      next += gridDim.x;
+      pre_blk[prefetched] = blk;
+      if (blk >= a.num_blocks) break;
+      issue_copies(prefetched++, blk);
+    }
+  }
+  grid_dependency_wait();
+  allow_dependent_launch();
 
   if (warp == 0) {
     // ---------------- producer warp ----------------
@@ -141,15 +187,24 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
     // whose completion the stage's barrier also tracks.
     int s = 0;
     uint32_t phase = 0;
-    long long next = blockIdx.x;
-    while (true) {
+    const int pre = __shfl_sync(0xffffffffu, prefetched, 0);
+    // A prefetch that ran into the end of the rows already took its terminating block.
+    const bool pre_ended = __shfl_sync(0xffffffffu, a.prefetch && prefetched < S ? 1 : 0, 0);
+    long long next = blockIdx.x + static_cast<long long>(pre) * gridDim.x;
+    for (int it = 0;; ++it) {
       long long blk = 0;
       bool ok = true;
+      const bool was_prefetched = it < pre;
       if (lane == 0) {
-        blk = a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
-        ok = mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty);
+        if (was_prefetched || (it == pre && pre_ended)) {
+          blk = pre_blk[it];
+        } else {
+          blk = a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull))
+                                   : next;
+          next += gridDim.x;
+        }
+        if (!was_prefetched) ok = mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty);
       }
-      next += gridDim.x;
       blk = __shfl_sync(0xffffffffu, blk, 0);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       __syncwarp();
@@ -166,11 +221,19 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
       uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
       if (lane == 0) {
         blk_id[s] = blk;
-        const uint32_t bytes = static_cast<uint32_t>(rows) * static_cast<uint32_t>(N) * 2u;
-        mbar_expect_tx(&full[s], 3u * bytes);
-        bulk_copy_g2s(st, a.dy + r0 * N, bytes, &full[s]);
-        bulk_copy_g2s(st + tensor_bytes, a.x + r0 * N, bytes, &full[s]);
-        bulk_copy_g2s(st + 2u * tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+        if (!was_prefetched) issue_copies(s, blk);
+        if (a.l2_prefetch && !a.dynamic_schedule) {
+          // the block this stage will hold next time round the ring
+          const long long ahead = blk + static_cast<long long>(S) * gridDim.x;
+          if (ahead < a.num_blocks) {
+            const long long aleft = a.M - ahead * R;
+            const uint32_t arows = static_cast<uint32_t>(aleft < R ? aleft : R);
+            const uint32_t abytes = arows * static_cast<uint32_t>(N) * 2u;
+            bulk_prefetch_l2(a.dy + ahead * R * N, abytes);
+            bulk_prefetch_l2(a.x + ahead * R * N, abytes);
+            bulk_prefetch_l2(a.g + ahead * R * N, abytes);
+          }
+        }
       }
       float* srs = reinterpret_cast<float*>(st + 3u * tensor_bytes);
       for (int i = lane; i < rows; i += 32) async_copy_4(srs + i, a.rstd + r0 + i);

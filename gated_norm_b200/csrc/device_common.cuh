@@ -91,6 +91,11 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
       : "memory");
 }
 
+// Warms L2 with `bytes` of global memory (no shared memory, registers or barrier involved).
+__device__ __forceinline__ void bulk_prefetch_l2(const void* gmem, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+}
+
 // Programmatic dependent launch: wait for the previous grid on the stream to complete
 // (and its memory to be visible) / allow the next grid to begin launching.
 __device__ __forceinline__ void grid_dependency_wait() {

@@ -49,33 +49,66 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
     fence_barrier_init();
   }
   __syncthreads();
-  grid_dependency_wait();     // inputs may come from the previous kernel on the stream
-  allow_dependent_launch();   // the next kernel may start its prologue on free SMs
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+
+  // Copies of stage s's block `blk` (x and g), counted on the stage's full barrier.
+  auto issue_copies = [&](int s, long long blk) {
+    const long long r0 = blk * R;
+    const long long left = a.M - r0;
+    const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
+    const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+    uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
+    mbar_expect_tx(&full[s], 2u * bytes);
+    bulk_copy_g2s(st, a.x + r0 * N, bytes, &full[s]);
+    bulk_copy_g2s(st + tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+  };
+
+  // When the host knows the previous kernel on the stream does not write x or g (the
+  // recompute forward of a checkpointed step), the first stages' copies start before that
+  // kernel has finished; nothing is written, and no stage is released to the consumers,
+  // before the dependency wait below.
+  int prefetched = 0;
+  if (a.prefetch && warp == 0 && lane == 0) {
+    for (long long blk = blockIdx.x; prefetched < S && blk < a.num_blocks; blk += gridDim.x)
+      issue_copies(prefetched++, blk);
+  }
+  grid_dependency_wait();     // inputs may come from the previous kernel on the stream
+  allow_dependent_launch();   // the next kernel may start its prologue on free SMs
 
   if (warp == 0) {
     // ---------------- producer: one lane issues the bulk copies ----------------
     if (lane == 0) {
       int s = 0;
       uint32_t phase = 0;
-      for (long long blk = blockIdx.x;; blk += gridDim.x) {
-        if (!mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty)) break;
-        if (blk >= a.num_blocks) {
-          blk_id[s] = -1;
+      int it = 0;
+      for (long long blk = blockIdx.x;; blk += gridDim.x, ++it) {
+        if (it < prefetched) {  // copies already in flight: publish the block
+          blk_id[s] = blk;
           mbar_arrive(&full[s]);
-          break;
+        } else {
+          if (!mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty)) break;
+          if (blk >= a.num_blocks) {
+            blk_id[s] = -1;
+            mbar_arrive(&full[s]);
+            break;
+          }
+          blk_id[s] = blk;
+          issue_copies(s, blk);
+          mbar_arrive(&full[s]);
+          if (a.l2_prefetch) {
+            // the block this stage will hold next time round the ring
+            const long long ahead = blk + static_cast<long long>(S) * gridDim.x;
+            if (ahead < a.num_blocks) {
+              const long long left = a.M - ahead * R;
+              const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
+              const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+              bulk_prefetch_l2(a.x + ahead * R * N, bytes);
+              bulk_prefetch_l2(a.g + ahead * R * N, bytes);
+            }
+          }
         }
-        blk_id[s] = blk;
-        const long long r0 = blk * R;
-        const long long left = a.M - r0;
-        const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
-        const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
-        uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
-        mbar_arrive_expect_tx(&full[s], 2u * bytes);
-        bulk_copy_g2s(st, a.x + r0 * N, bytes, &full[s]);
-        bulk_copy_g2s(st + tensor_bytes, a.g + r0 * N, bytes, &full[s]);
         if (++s == S) {
           s = 0;
           phase ^= 1u;

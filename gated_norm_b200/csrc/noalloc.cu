@@ -137,6 +137,8 @@ extern "C" int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, c
   a.dynamic_schedule = plan.dynamic_schedule;
   a.fused_reduce = plan.fused_reduce;
   a.dw_fp32 = dw_fp32 ? 1 : 0;
+  a.prefetch = 0;
+  a.l2_prefetch = plan.l2_prefetch;
   a.err = reinterpret_cast<unsigned*>(sc.ptr + kStaticErrWordOffset);
   const bool pdl = get_tuning().disable_pdl == 0;
   if (launch_bwd(plan, a, s, pdl) != cudaSuccess) return GNORM_ERR_CUDA;

@@ -21,7 +21,7 @@
 
 namespace gnorm {
 
-static TuningKnobs g_knobs;  // all zero: built-in values
+static TuningKnobs g_knobs = {};  // all zero: built-in values
 
 void set_tuning(const TuningKnobs& k) { g_knobs = k; }
 TuningKnobs get_tuning() { return g_knobs; }
@@ -142,15 +142,16 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   out->grid = static_cast<int>(grid);
   out->num_blocks = blocks;
   out->smem_bytes = static_cast<int>(smem);
+  out->l2_prefetch = g_knobs.l2_prefetch == 1 ? 1 : (g_knobs.l2_prefetch == 2 ? 0 : kDefaultL2Prefetch);
   if (kind == 1) {
     out->dynamic_schedule = deterministic ? 0 : 1;
     out->partials = static_cast<int>(grid);
-    // The last-CTA tail pays off when the partials are small; wide rows use the second
-    // launch, whose CTAs read the partials in parallel.
+    // The fixed-order second pass over the partials runs in the last CTA to finish when the
+    // partials are small (one launch; the result does not depend on which CTA is last),
+    // and as a second launch whose CTAs read them in parallel for wide rows.
+    const int tail = g_knobs.tail_reduce == 1 ? 1 : (g_knobs.tail_reduce == 2 ? 0 : kDefaultTailReduce);
     out->fused_reduce =
-        (!deterministic && grid > 0 && static_cast<int64_t>(grid) * N <= kFusedReduceMaxFloats)
-            ? 1
-            : 0;
+        (tail && grid > 0 && static_cast<int64_t>(grid) * N <= kFusedReduceMaxFloats) ? 1 : 0;
   }
   return GNORM_OK;
 }

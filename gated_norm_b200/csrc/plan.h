@@ -23,6 +23,17 @@ constexpr int64_t kFwdLatencyStageBytes = 16384;
 constexpr int64_t kFwdLatencyTierBytes = 512 * 1024;
 constexpr int64_t kBwdStageBytes = 49152;
 constexpr int kBwdMinStageRows = 3;
+// Measured on B200 in same-box A/B runs (graph replays, cold L2):
+//  * an L2 bulk prefetch of the block after each CTA's ring slows every workload (e.g.
+//    368640x128 forward 55 -> 68 us, backward 86 -> 113 us): off;
+//  * the dw second pass as a second (programmatic-dependent) launch is as fast as or faster
+//    than running it in the backward's last CTA (e.g. 262144x256 backward 118.8 vs 121 us):
+//    second launch by default;
+//  * letting gnorm_ckpt_step's recompute forward and backward copy their inputs before the
+//    previous kernel ends saves 3-6 us per step (e.g. 16384x4096 241 -> 235.5 us): on.
+constexpr int kDefaultL2Prefetch = 0;
+constexpr int kDefaultTailReduce = 0;
+constexpr int kDefaultChainPrefetch = 1;
 constexpr int64_t kFusedReduceMaxFloats = 65536;
 
 struct RowGeometry {
@@ -30,21 +41,14 @@ struct RowGeometry {
   int chunks_per_thread;
 };
 
-// Experiment knobs (0 = built-in value).  Process-wide; not used unless set.
-struct TuningKnobs {
-  int stage_bytes;
-  int max_stages;
-  int ctas_per_sm;
-  int disable_pdl;
-  int threads_per_row;    // with chunks_per_thread: force a compiled row geometry
-  int chunks_per_thread;
-};
-
-// Row geometries with compiled kernels, per kind (0 forward, 1 backward).
-bool geometry_compiled(int kind, int threads_per_row, int chunks_per_thread);
+// Experiment knobs (gnorm_tuning of include/gnorm.h; 0 = built-in value).  Process-wide.
+using TuningKnobs = gnorm_tuning;
 
 void set_tuning(const TuningKnobs& k);
 TuningKnobs get_tuning();
+
+// Row geometries with compiled kernels, per kind (0 forward, 1 backward).
+bool geometry_compiled(int kind, int threads_per_row, int chunks_per_thread);
 
 RowGeometry geometry_for(int64_t N);
 int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,

@@ -12,7 +12,7 @@ import threading
 
 import torch
 
-from ._lib import GNORM_OK, GnormPlan, lib
+from ._lib import GNORM_OK, GnormPlan, GnormTuning, lib
 
 __all__ = [
     "GnormError",
@@ -70,11 +70,17 @@ def gnorm_device_error(reset: bool = False) -> int:
     return int(lib.gnorm_device_error(int(bool(reset))))
 
 
-def gnorm_set_tuning(stage_bytes: int = 0, max_stages: int = 0, ctas_per_sm: int = 0,
-                     disable_pdl: bool = False, threads_per_row: int = 0,
-                     chunks_per_thread: int = 0) -> None:
-    lib.gnorm_set_tuning(int(stage_bytes), int(max_stages), int(ctas_per_sm),
-                         int(bool(disable_pdl)), int(threads_per_row), int(chunks_per_thread))
+def gnorm_set_tuning(**knobs) -> None:
+    """Process-wide experiment knobs (fields of gnorm_tuning; 0 = built-in).  No arguments
+    restores every built-in choice.  Tri-state knobs (l2_prefetch, tail_reduce,
+    chain_prefetch): 1 on, 2 off, 0 built-in."""
+    t = GnormTuning()
+    names = {f for f, _ in GnormTuning._fields_}
+    for k, v in knobs.items():
+        if k not in names:
+            raise TypeError(f"unknown tuning knob {k!r}")
+        setattr(t, k, int(v))
+    lib.gnorm_set_tuning(ctypes.byref(t) if knobs else None)
 
 
 # ----------------------------------------------------------------------------- helpers

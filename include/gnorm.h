@@ -81,9 +81,11 @@ GNORM_API int gnorm_fwd(const void* x, const void* g, const void* w, float eps,
  * Flashinfer PR #8701, section "How the tables were measured": "bwdg" (BF16 dw) and
  * "bwdg_f32" (FP32 dw); the deterministic package is the same API with deterministic=True.
  *
- * deterministic != 0: rows are assigned to CTAs by a fixed rule and the FP32 dw partials are
- *   summed in a fixed order by a second launch, so dx, dg and dw are bitwise identical from
- *   run to run on the same device model with the same arguments.
+ * Each CTA sums its rows' dw terms in FP32 into one partial row; a second pass sums the
+ * partials in a fixed order in a second launch (or, when the tail_reduce knob asks and
+ * partials x N <= 65536, in the backward's last CTA to finish).
+ * deterministic != 0: rows are assigned to CTAs by a fixed rule, so dx, dg and dw are
+ *   bitwise identical from run to run on the same device model with the same arguments.
  * deterministic == 0: CTAs take row blocks from a shared counter, so dw's FP32 summation
  *   order can change between runs (dx and dg do not); dw is never accumulated with float
  *   atomics.
@@ -174,7 +176,7 @@ typedef struct gnorm_plan {
   int dynamic_schedule;  /* 1: CTAs take row blocks from an atomic counter */
   int fused_reduce;      /* 1: the last CTA to finish reduces the dw partials */
   int partials;          /* rows of the FP32 dw partial buffer (backward), else 0 */
-  int reserved;
+  int l2_prefetch;       /* 1: warm L2 with the block each CTA loads after its ring's */
 } gnorm_plan;
 
 /*
@@ -194,15 +196,23 @@ GNORM_API int gnorm_plan_query(int kind, int64_t M, int64_t N, int deterministic
 GNORM_API int gnorm_device_error(int reset);
 
 /*
- * Process-wide tuning knobs for experiments (0 keeps the built-in value): target bytes per
- * pipeline stage, maximum pipeline depth, resident CTAs per SM, 1 to launch without
- * programmatic dependent launch, and a forced row geometry (threads per row and 16-byte
- * chunks per thread; both must name a compiled geometry that covers N, else plans fail
- * with GNORM_ERR_UNSUPPORTED).  Affects plans made after the call, including
- * gnorm_plan_query and gnorm_bwd_workspace_bytes.  Not thread-safe with concurrent calls.
+ * Process-wide tuning knobs for experiments.  Every field 0 keeps the built-in choice.
+ * Affects plans and launches made after the call (including gnorm_plan_query and
+ * gnorm_bwd_workspace_bytes); not thread-safe with concurrent calls.  NULL resets all.
  */
-GNORM_API void gnorm_set_tuning(int stage_bytes, int max_stages, int ctas_per_sm, int disable_pdl,
-                                int threads_per_row, int chunks_per_thread);
+typedef struct gnorm_tuning {
+  int stage_bytes;       /* target bytes per pipeline stage */
+  int max_stages;        /* maximum pipeline depth */
+  int ctas_per_sm;       /* resident CTAs per SM (capped by the kernel's compiled residency) */
+  int disable_pdl;       /* 1: launch without programmatic dependent launch */
+  int threads_per_row;   /* with chunks_per_thread: force a compiled row geometry covering N, */
+  int chunks_per_thread; /*   else plans fail with GNORM_ERR_UNSUPPORTED */
+  int l2_prefetch;       /* 1: warm L2 with the block after each CTA's ring, 2: do not */
+  int tail_reduce;       /* 1: dw second pass in the backward's last CTA when small, 2: never */
+  int chain_prefetch;    /* 1: in gnorm_ckpt_step, copy inputs before the previous kernel ends, 2: do not */
+} gnorm_tuning;
+
+GNORM_API void gnorm_set_tuning(const gnorm_tuning* tuning);
 
 /* Build description: compiler version, target architecture (static storage). */
 GNORM_API const char* gnorm_build_info(void);

@@ -100,8 +100,7 @@ def test_plan_invariants(sms, kind):
                     assert p["smem_bytes"] >= 1024 + groups * N * 4 + p["consumer_threads"] * 16
                     assert p["partials"] == G
                     assert p["dynamic_schedule"] == (0 if det else 1)
-                    if det:
-                        assert p["fused_reduce"] == 0
+                    assert p["fused_reduce"] == 0  # second launch unless the knob asks
 
 
 def test_plan_is_a_pure_function():
@@ -213,3 +212,19 @@ def test_forced_geometry_knob():
             gn.gnorm_plan_query(0, 64, 128, True, 148)
     finally:
         gn.gnorm_set_tuning()
+
+
+def test_tail_and_l2_knobs_in_plans():
+    base = gn.gnorm_plan_query(1, 65536, 128, True, 148)
+    assert base["fused_reduce"] == 0 and base["l2_prefetch"] == 0
+    try:
+        gn.gnorm_set_tuning(tail_reduce=1, l2_prefetch=1)
+        p = gn.gnorm_plan_query(1, 65536, 128, True, 148)
+        assert p["fused_reduce"] == 1 and p["l2_prefetch"] == 1
+        gn.gnorm_set_tuning(tail_reduce=1)
+        assert gn.gnorm_plan_query(1, 65536, 4096, True, 148)["fused_reduce"] == 0  # too big
+        with pytest.raises(TypeError):
+            gn.gnorm_set_tuning(no_such_knob=1)
+    finally:
+        gn.gnorm_set_tuning()
+    assert gn.gnorm_plan_query(1, 65536, 128, True, 148) == base

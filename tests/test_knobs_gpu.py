@@ -1,0 +1,56 @@
+"""Every tuning knob keeps the results right (GPU).
+
+The knobs change launch shapes, pipeline depth, where the dw second pass runs, and whether
+inputs are prefetched; y, rstd, dx and dg must not change at all (they are per row), and
+dw must stay within its tolerance of the oracle.
+"""
+from __future__ import annotations
+
+import itertools
+
+import pytest
+import torch
+
+from gpu_util import Case, dev_to_f64
+from tolerance import dw_fp32_check
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    import gated_norm_b200 as gn
+
+KNOB_SETS = [
+    dict(tail_reduce=t, chain_prefetch=c, l2_prefetch=l)
+    for t, c, l in itertools.product((1, 2), (1, 2), (1, 2))
+] + [
+    dict(disable_pdl=1),
+    dict(ctas_per_sm=1, stage_bytes=8192, max_stages=2),
+    dict(ctas_per_sm=2, stage_bytes=98304),
+]
+
+
+@pytest.mark.parametrize("M,N", [(4099, 128), (700, 4096), (2500, 256)])
+@pytest.mark.parametrize("det", [True, False])
+def test_knobs_do_not_change_results(M, N, det):
+    case = Case(M, N, seed=23)
+    ref = gn.gnorm_ckpt_step(case.x, case.g, case.w, case.eps, case.dy, dw_fp32=True,
+                             deterministic=det)
+    torch.cuda.synchronize()
+    dw_oracle = case.oracle_dw()
+    try:
+        for knobs in KNOB_SETS:
+            gn.gnorm_set_tuning(**knobs)
+            out = gn.gnorm_ckpt_step(case.x, case.g, case.w, case.eps, case.dy, dw_fp32=True,
+                                     deterministic=det)
+            dx2, dg2, dw2 = gn.gnorm_bwd(case.dy, case.x, case.g, case.w, out[1], dw_fp32=True,
+                                         deterministic=det)
+            torch.cuda.synchronize()
+            for a, b, name in zip(ref[:4], out[:4], ("y", "rstd", "dx", "dg")):
+                assert torch.equal(a, b), (knobs, name)
+            assert torch.equal(dx2, ref[2]) and torch.equal(dg2, ref[3]), knobs
+            for dw in (out[4], dw2):
+                rep = dw_fp32_check(dev_to_f64(dw), dw_oracle)
+                assert rep["ok"], (knobs, rep)
+    finally:
+        gn.gnorm_set_tuning()
+    assert gn.gnorm_device_error(reset=True) == 0
