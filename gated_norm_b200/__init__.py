@@ -16,6 +16,7 @@ from .gnorm import (  # noqa: F401
     gnorm_dw_reduce,
     gnorm_fwd,
     gnorm_plan_query,
+    gnorm_selftest_wait_timeout,
     gnorm_set_tuning,
     gnorm_status_string,
     workspace,

@@ -55,6 +55,38 @@ class GnormTuning(ctypes.Structure):
         "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch")]
 
 
+class GnormFwdDesc(ctypes.Structure):
+    """Mirror of ``gnorm_fwd_desc`` in include/gnorm.h."""
+
+    _fields_ = [
+        ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
+        ("g", ctypes.c_void_p), ("ldg", ctypes.c_int64),
+        ("w", ctypes.c_void_p), ("w_fp32", ctypes.c_int),
+        ("eps", ctypes.c_float),
+        ("y", ctypes.c_void_p), ("ldy", ctypes.c_int64),
+        ("rstd", ctypes.c_void_p),
+        ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+    ]
+
+
+class GnormBwdDesc(ctypes.Structure):
+    """Mirror of ``gnorm_bwd_desc`` in include/gnorm.h."""
+
+    _fields_ = [
+        ("dy", ctypes.c_void_p), ("lddy", ctypes.c_int64),
+        ("x", ctypes.c_void_p), ("ldx", ctypes.c_int64),
+        ("g", ctypes.c_void_p), ("ldg", ctypes.c_int64),
+        ("w", ctypes.c_void_p), ("w_fp32", ctypes.c_int),
+        ("rstd", ctypes.c_void_p),
+        ("dx", ctypes.c_void_p), ("lddx", ctypes.c_int64),
+        ("dg", ctypes.c_void_p), ("lddg", ctypes.c_int64),
+        ("dw", ctypes.c_void_p), ("dw_fp32", ctypes.c_int),
+        ("deterministic", ctypes.c_int),
+        ("M", ctypes.c_int64), ("N", ctypes.c_int64),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_size_t),
+    ]
+
+
 _vp = ctypes.c_void_p
 _i64 = ctypes.c_int64
 _int = ctypes.c_int
@@ -68,6 +100,9 @@ SIGNATURES = {
                          _vp]),
     "gnorm_bwd_noalloc": (_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _i64,
                                  _vp]),
+    "gnorm_fwd_ex": (_int, [ctypes.POINTER(GnormFwdDesc), _vp]),
+    "gnorm_bwd_ex": (_int, [ctypes.POINTER(GnormBwdDesc), _vp]),
+    "gnorm_ckpt_step_ex": (_int, [ctypes.POINTER(GnormFwdDesc), ctypes.POINTER(GnormBwdDesc), _vp]),
     "gnorm_ckpt_step": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
                                _i64, _vp, _sz, _vp]),
     "gnorm_dw_reduce": (_int, [_vp, _i64, _i64, _vp, _int, _vp]),
@@ -76,6 +111,7 @@ SIGNATURES = {
     "gnorm_status_string": (ctypes.c_char_p, [_int]),
     "gnorm_plan_query": (_int, [_int, _i64, _i64, _int, _int, _int, ctypes.POINTER(GnormPlan)]),
     "gnorm_device_error": (_int, [_int]),
+    "gnorm_selftest_wait_timeout": (_int, [ctypes.c_uint, ctypes.POINTER(ctypes.c_ulonglong)]),
     "gnorm_set_tuning": (None, [ctypes.POINTER(GnormTuning)]),
     "gnorm_build_info": (ctypes.c_char_p, []),
 }

@@ -1,16 +1,24 @@
 // args.h -- kernel argument blocks (plain structs shared by host and device code).
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
 #include <stdint.h>
 
 namespace gnorm {
 
+// Row strides (ld*) are in elements; a tensor with ld == N is packed.  A strided tensor may
+// also come with a 2-D tiled tensor map (box = N columns x rows_per_stage rows) that loads a
+// whole row block in one copy; map_bits says which maps are valid.
 struct FwdArgs {
+  CUtensorMap map_x, map_g;
+  int map_bits = 0;  // bit 0: map_x, bit 1: map_g
   const uint16_t* x;
   const uint16_t* g;
-  const uint16_t* w;
+  const void* w;  // BF16 or FP32 [N] (w_fp32)
   uint16_t* y;
   float* rstd;
+  long long ldx = 0, ldg = 0, ldy = 0;
+  int w_fp32 = 0;
   long long M;
   int N;
   float eps;
@@ -24,13 +32,17 @@ struct FwdArgs {
 };
 
 struct BwdArgs {
+  CUtensorMap map_dy, map_x, map_g;
+  int map_bits = 0;  // bit 0: map_dy, bit 1: map_x, bit 2: map_g
   const uint16_t* dy;
   const uint16_t* x;
   const uint16_t* g;
-  const uint16_t* w;
+  const void* w;  // BF16 or FP32 [N] (w_fp32)
   const float* rstd;
   uint16_t* dx;
   uint16_t* dg;
+  long long lddy = 0, ldx = 0, ldg = 0, lddx = 0, lddg = 0;
+  int w_fp32 = 0;
   float* partial;                    // [gridDim.x, N] FP32 dw partials (workspace)
   void* dw;                          // written by the fused tail only
   unsigned long long* work_counter;  // dynamic schedule (workspace header)

@@ -10,7 +10,7 @@
 // reduced in a fixed order.)
 //
 // Design: the same persistent, warp-specialised TMA pipeline as the forward, with three
-// tensors (dy, x, g) per stage.  Pass 1 recomputes xhat and the gate from shared memory,
+// tensors (dy, x, g) per stage (packed or strided rows).  Pass 1 recomputes xhat and the gate from shared memory,
 // writes dg, accumulates the row dot product sum(u xhat) and this thread's dw columns in
 // FP32 registers (arithmetic on packed FP32 pairs), and keeps u in registers; after the row
 // reduction pass 2 re-reads x and writes dx.  The producer warp also stages the rows' rstd
@@ -102,7 +102,8 @@ __device__ __forceinline__ void reduce_partials(const float* __restrict__ partia
   }
 }
 
-// Second pass over the dw partials (both modes): one CTA per 128 columns.
+// Second pass over the dw partials (both modes): one 1024-thread CTA per 128 columns, so
+// 32 lanes share the partial rows and each issues all its loads at once for P <= 256.
 // Also clears the dynamic-schedule counter of the workspace (the backward grid has
 // finished by now).
 __global__ void __launch_bounds__(kReduceThreads)
@@ -118,7 +119,7 @@ __global__ void __launch_bounds__(kReduceThreads)
 
 template <int TPR, int CPT>
 __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(1, TPR, CPT))
-    gated_rmsnorm_bwd_kernel(const BwdArgs a) {
+    gated_rmsnorm_bwd_kernel(const __grid_constant__ BwdArgs a) {
   constexpr int kNCT = consumer_threads_for(TPR);
   constexpr int kGroups = kNCT / TPR;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -132,7 +133,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   const int S = a.stages;
   const int R = a.rows_per_stage;
   const int N = a.N;
-  const uint32_t tensor_bytes = static_cast<uint32_t>(R) * N * 2u;
+  const uint32_t tensor_bytes = static_cast<uint32_t>(stage_tensor_bytes(R, N));
   const uint32_t stage_bytes = (3u * tensor_bytes + static_cast<uint32_t>(R) * 4u + 127u) & ~127u;
 
   if (threadIdx.x == 0) {
@@ -148,17 +149,21 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Bulk copies of stage s's block `blk` (dy, x, g), counted on the stage's full barrier.
+  // Bulk copies of stage s's block `blk` (dy, x, g) by the producer warp's lanes, counted on
+  // the stage's full barrier (lane 0 posts the byte count first).
   auto issue_copies = [&](int s, long long blk) {
     const long long r0 = blk * R;
     const long long left = a.M - r0;
-    const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
-    const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+    const int rows = static_cast<int>(left < R ? left : R);
     uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
-    mbar_expect_tx(&full[s], 3u * bytes);
-    bulk_copy_g2s(st, a.dy + r0 * N, bytes, &full[s]);
-    bulk_copy_g2s(st + tensor_bytes, a.x + r0 * N, bytes, &full[s]);
-    bulk_copy_g2s(st + 2u * tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+    if (lane == 0) mbar_expect_tx(&full[s], 3u * static_cast<uint32_t>(rows) * N * 2u);
+    __syncwarp();
+    copy_row_block(st, a.dy, a.lddy, N, r0, rows, R, (a.map_bits & 1) ? &a.map_dy : nullptr,
+                   &full[s], lane);
+    copy_row_block(st + tensor_bytes, a.x, a.ldx, N, r0, rows, R,
+                   (a.map_bits & 2) ? &a.map_x : nullptr, &full[s], lane);
+    copy_row_block(st + 2u * tensor_bytes, a.g, a.ldg, N, r0, rows, R,
+                   (a.map_bits & 4) ? &a.map_g : nullptr, &full[s], lane);
   };
 
   // When the host knows the previous kernel on the stream writes none of dy, x, g (the
@@ -166,11 +171,13 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   // finished.  rstd, which that forward writes, is copied only after the wait below.
   int prefetched = 0;
   long long pre_blk[kMaxStages];
-  if (a.prefetch && warp == 0 && lane == 0) {
+  if (a.prefetch && warp == 0) {
     long long next = blockIdx.x;
     while (prefetched < S) {
-      const long long blk =
-          a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
+      long long blk = 0;
+      if (lane == 0)
+        blk = a.dynamic_schedule ? static_cast<long long>(atomicAdd(a.work_counter, 1ull)) : next;
+      blk = __shfl_sync(0xffffffffu, blk, 0);
       next += gridDim.x;
       pre_blk[prefetched] = blk;
       if (blk >= a.num_blocks) break;
@@ -182,14 +189,14 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
 
   if (warp == 0) {
     // ---------------- producer warp ----------------
-    // Lane 0 takes the next row block, waits for a free stage and issues the bulk copies of
-    // dy, x and g; all 32 lanes copy the block's rstd values with 4-byte asynchronous copies
+    // Lane 0 takes the next row block and waits for a free stage; the lanes issue the bulk
+    // copies of dy, x and g and copy the block's rstd values with 4-byte asynchronous copies
     // whose completion the stage's barrier also tracks.
     int s = 0;
     uint32_t phase = 0;
-    const int pre = __shfl_sync(0xffffffffu, prefetched, 0);
+    const int pre = prefetched;  // the same in every lane of this warp
     // A prefetch that ran into the end of the rows already took its terminating block.
-    const bool pre_ended = __shfl_sync(0xffffffffu, a.prefetch && prefetched < S ? 1 : 0, 0);
+    const bool pre_ended = a.prefetch && prefetched < S;
     long long next = blockIdx.x + static_cast<long long>(pre) * gridDim.x;
     for (int it = 0;; ++it) {
       long long blk = 0;
@@ -219,10 +226,10 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
       const long long left = a.M - r0;
       const int rows = static_cast<int>(left < R ? left : R);
       uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
+      if (!was_prefetched) issue_copies(s, blk);
       if (lane == 0) {
         blk_id[s] = blk;
-        if (!was_prefetched) issue_copies(s, blk);
-        if (a.l2_prefetch && !a.dynamic_schedule) {
+        if (a.l2_prefetch && !a.dynamic_schedule && a.lddy == N && a.ldx == N && a.ldg == N) {
           // the block this stage will hold next time round the ring
           const long long ahead = blk + static_cast<long long>(S) * gridDim.x;
           if (ahead < a.num_blocks) {
@@ -265,7 +272,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
       wp[k][i] = splat2(0.f);
       dwacc[k][i] = splat2(0.f);
     }
-    if (cval[k]) bf16x8_to_pairs(*reinterpret_cast<const uint4*>(a.w + c * 8), wp[k]);
+    if (cval[k]) load_weight_pairs(a.w, a.w_fp32, c, wp[k]);
   }
 
   int s = 0;
@@ -319,7 +326,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
             dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), dsilu);
           }
           if (valid)
-            *reinterpret_cast<uint4*>(a.dg + grow * N + c * 8) = pairs_to_bf16x8(dgp);
+            *reinterpret_cast<uint4*>(a.dg + grow * a.lddg + c * 8) = pairs_to_bf16x8(dgp);
         }
       }
       const float dot = row_sum<TPR>(dot2.x + dot2.y, red_slots, group, lr, slot);
@@ -339,7 +346,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
           for (int i = 0; i < 4; ++i)
             dxp[i] = fma2(nrc2, mul2(xp[i], r2), mul2(r2, u[k][i]));
           if (valid)
-            *reinterpret_cast<uint4*>(a.dx + grow * N + c * 8) = pairs_to_bf16x8(dxp);
+            *reinterpret_cast<uint4*>(a.dx + grow * a.lddx + c * 8) = pairs_to_bf16x8(dxp);
         }
       }
     }

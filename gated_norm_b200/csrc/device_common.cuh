@@ -3,6 +3,7 @@
 // programmatic dependent launch, BF16 packing and the logistic function.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -14,6 +15,7 @@ namespace gnorm {
 // Bits of the device error word (see gnorm_device_error in include/gnorm.h).
 constexpr unsigned kErrWaitFull = 1u;   // a consumer gave up waiting for copied rows
 constexpr unsigned kErrWaitEmpty = 2u;  // the producer gave up waiting for a free stage
+constexpr unsigned kErrSelfTest = 4u;   // the self-test's wait ran out, as it should
 
 // A pipeline wait that has not completed after this long is abandoned.  A stage of a
 // few tens of KB arrives in microseconds, so two seconds only trips on a real fault.
@@ -65,7 +67,8 @@ __device__ __forceinline__ unsigned long long globaltimer_ns() {
 // kWaitLimitNs (or 2^24 polling rounds, whichever comes first), sets `err_bit` in the
 // device error word and returns false; the caller then stops its loop and exits.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err_word,
-                                          unsigned err_bit) {
+                                          unsigned err_bit,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
@@ -73,7 +76,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(a, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    if (globaltimer_ns() - t0 > limit_ns) break;
   }
   atomicOr(err_word, err_bit);
   return false;
@@ -88,6 +91,17 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
           "r"(smem_u32(smem_dst)),
       "l"(gmem_src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Tiled 2-D TMA load of the box at (c0, c1) of `map` into shared memory (128-byte aligned),
+// completion counted in bytes on `bar`.  No multicast.
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
       : "memory");
 }
 
@@ -225,6 +239,41 @@ __device__ __forceinline__ float row_sum(float v, float* red_slots, int group, i
     for (int i = 1; i < kWarps; ++i) v += slots[i];
   }
   return v;
+}
+
+// Rows [r0, r0 + rows) of a tensor with row stride `ld` elements into shared memory as packed
+// rows of N BF16 values.  Packed rows (ld == N) are one bulk copy issued by lane 0; strided
+// rows are one bulk copy per row, spread over the warp's 32 lanes.  Every byte lands on
+// `bar`, whose expected byte count the caller has already posted.
+// A full block of a strided tensor that has a 2-D tiled tensor map (box N x R) is one tiled
+// copy at coordinates (column 0, row r0): the innermost coordinate is 0, so 16-byte aligned.
+__device__ __forceinline__ void copy_row_block(uint8_t* dst, const uint16_t* src, long long ld,
+                                               int N, long long r0, int rows, int R,
+                                               const CUtensorMap* map, uint64_t* bar,
+                                               int lane) {
+  const uint32_t row_bytes = static_cast<uint32_t>(N) * 2u;
+  if (ld == N) {
+    if (lane == 0) bulk_copy_g2s(dst, src + r0 * N, static_cast<uint32_t>(rows) * row_bytes, bar);
+  } else if (map != nullptr && rows == R) {
+    if (lane == 0) tma_load_2d(dst, map, 0, static_cast<int>(r0), bar);
+  } else {
+    for (int i = lane; i < rows; i += 32)
+      bulk_copy_g2s(dst + static_cast<size_t>(i) * row_bytes, src + (r0 + i) * ld, row_bytes, bar);
+  }
+}
+
+// This thread's 8 weights of chunk c as FP32 pairs, from a BF16 or FP32 weight vector.
+__device__ __forceinline__ void load_weight_pairs(const void* w, int w_fp32, int c, float2 p[4]) {
+  if (w_fp32) {
+    const float4* w4 = reinterpret_cast<const float4*>(w) + 2 * c;
+    const float4 a = w4[0], b = w4[1];
+    p[0] = make_float2(a.x, a.y);
+    p[1] = make_float2(a.z, a.w);
+    p[2] = make_float2(b.x, b.y);
+    p[3] = make_float2(b.z, b.w);
+  } else {
+    bf16x8_to_pairs(reinterpret_cast<const uint4*>(w)[c], p);
+  }
 }
 
 }  // namespace gnorm

@@ -6,10 +6,10 @@
 // of "Cake's SiLU-gated RMSNorm training kernel"; the pages print no kernel, so the design
 // below is this library's own.)
 //
-// Design: a persistent, warp-specialised CTA.  Warp 0 (one elected lane) streams row
-// blocks of x and g from HBM into a ring of shared-memory stages with 1-D TMA bulk copies
-// (rows are packed, so a block of R rows of one tensor is one contiguous copy) and
-// mbarrier transaction counts.  The consumer warps own `TPR` threads per row and `CPT`
+// Design: a persistent, warp-specialised CTA.  Warp 0 streams row blocks of x and g from
+// HBM into a ring of shared-memory stages with 1-D TMA bulk copies and mbarrier transaction
+// counts (packed rows: a block of R rows of one tensor is one contiguous copy; strided rows:
+// one copy per row, spread over the warp's lanes).  The consumer warps own `TPR` threads per row and `CPT`
 // 16-byte chunks per thread: pass 1 reads x from shared memory and reduces the sum of
 // squares (shuffles, plus named-barrier slots when a row spans several warps); pass 2
 // reads g and writes y straight to HBM with 16-byte stores.  Row blocks are assigned
@@ -24,7 +24,7 @@ namespace gnorm {
 
 template <int TPR, int CPT>
 __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(0, TPR, CPT))
-    gated_rmsnorm_fwd_kernel(const FwdArgs a) {
+    gated_rmsnorm_fwd_kernel(const __grid_constant__ FwdArgs a) {
   constexpr int kNCT = consumer_threads_for(TPR);
   constexpr int kGroups = kNCT / TPR;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -37,7 +37,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   const int S = a.stages;
   const int R = a.rows_per_stage;
   const int N = a.N;
-  const uint32_t tensor_bytes = static_cast<uint32_t>(R) * N * 2u;  // one tensor of a stage
+  const uint32_t tensor_bytes = static_cast<uint32_t>(stage_tensor_bytes(R, N));  // one tensor of a stage
   const uint32_t stage_bytes = (2u * tensor_bytes + 127u) & ~127u;
   constexpr int num_consumer_warps = kNCT / 32;
 
@@ -53,16 +53,19 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Copies of stage s's block `blk` (x and g), counted on the stage's full barrier.
+  // Copies of stage s's block `blk` (x and g) by the producer warp's lanes, counted on the
+  // stage's full barrier (lane 0 posts the byte count first).
   auto issue_copies = [&](int s, long long blk) {
     const long long r0 = blk * R;
     const long long left = a.M - r0;
-    const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
-    const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+    const int rows = static_cast<int>(left < R ? left : R);
     uint8_t* st = stage0 + static_cast<size_t>(s) * stage_bytes;
-    mbar_expect_tx(&full[s], 2u * bytes);
-    bulk_copy_g2s(st, a.x + r0 * N, bytes, &full[s]);
-    bulk_copy_g2s(st + tensor_bytes, a.g + r0 * N, bytes, &full[s]);
+    if (lane == 0) mbar_expect_tx(&full[s], 2u * static_cast<uint32_t>(rows) * N * 2u);
+    __syncwarp();
+    copy_row_block(st, a.x, a.ldx, N, r0, rows, R, (a.map_bits & 1) ? &a.map_x : nullptr,
+                   &full[s], lane);
+    copy_row_block(st + tensor_bytes, a.g, a.ldg, N, r0, rows, R,
+                   (a.map_bits & 2) ? &a.map_g : nullptr, &full[s], lane);
   };
 
   // When the host knows the previous kernel on the stream does not write x or g (the
@@ -70,7 +73,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   // kernel has finished; nothing is written, and no stage is released to the consumers,
   // before the dependency wait below.
   int prefetched = 0;
-  if (a.prefetch && warp == 0 && lane == 0) {
+  if (a.prefetch && warp == 0) {
     for (long long blk = blockIdx.x; prefetched < S && blk < a.num_blocks; blk += gridDim.x)
       issue_copies(prefetched++, blk);
   }
@@ -78,41 +81,45 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
   allow_dependent_launch();   // the next kernel may start its prologue on free SMs
 
   if (warp == 0) {
-    // ---------------- producer: one lane issues the bulk copies ----------------
-    if (lane == 0) {
-      int s = 0;
-      uint32_t phase = 0;
-      int it = 0;
-      for (long long blk = blockIdx.x;; blk += gridDim.x, ++it) {
-        if (it < prefetched) {  // copies already in flight: publish the block
-          blk_id[s] = blk;
-          mbar_arrive(&full[s]);
-        } else {
-          if (!mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty)) break;
-          if (blk >= a.num_blocks) {
+    // ---------------- producer warp ----------------
+    // Lane 0 waits for a free stage and publishes the block; the lanes issue its copies.
+    int s = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    for (long long blk = blockIdx.x;; blk += gridDim.x, ++it) {
+      if (it >= prefetched) {
+        bool ok = true;
+        if (lane == 0) ok = mbar_wait(&empty[s], phase ^ 1u, a.err, kErrWaitEmpty);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        __syncwarp();
+        if (!ok) break;
+        if (blk >= a.num_blocks) {
+          if (lane == 0) {
             blk_id[s] = -1;
             mbar_arrive(&full[s]);
-            break;
           }
-          blk_id[s] = blk;
-          issue_copies(s, blk);
-          mbar_arrive(&full[s]);
-          if (a.l2_prefetch) {
-            // the block this stage will hold next time round the ring
-            const long long ahead = blk + static_cast<long long>(S) * gridDim.x;
-            if (ahead < a.num_blocks) {
-              const long long left = a.M - ahead * R;
-              const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
-              const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
-              bulk_prefetch_l2(a.x + ahead * R * N, bytes);
-              bulk_prefetch_l2(a.g + ahead * R * N, bytes);
-            }
+          break;
+        }
+        issue_copies(s, blk);
+        if (a.l2_prefetch && a.ldx == N && a.ldg == N && lane == 0) {
+          // the block this stage will hold next time round the ring
+          const long long ahead = blk + static_cast<long long>(S) * gridDim.x;
+          if (ahead < a.num_blocks) {
+            const long long left = a.M - ahead * R;
+            const uint32_t rows = static_cast<uint32_t>(left < R ? left : R);
+            const uint32_t bytes = rows * static_cast<uint32_t>(N) * 2u;
+            bulk_prefetch_l2(a.x + ahead * R * N, bytes);
+            bulk_prefetch_l2(a.g + ahead * R * N, bytes);
           }
         }
-        if (++s == S) {
-          s = 0;
-          phase ^= 1u;
-        }
+      }
+      if (lane == 0) {  // publish the block (its copies are in flight)
+        blk_id[s] = blk;
+        mbar_arrive(&full[s]);
+      }
+      if (++s == S) {
+        s = 0;
+        phase ^= 1u;
       }
     }
     return;
@@ -132,7 +139,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
     cval[k] = c < n8;
 #pragma unroll
     for (int i = 0; i < 4; ++i) wp[k][i] = splat2(0.f);
-    if (cval[k]) bf16x8_to_pairs(*reinterpret_cast<const uint4*>(a.w + c * 8), wp[k]);
+    if (cval[k]) load_weight_pairs(a.w, a.w_fp32, c, wp[k]);
   }
 
   int s = 0;
@@ -189,7 +196,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
             yp[i] = mul2(mul2(mul2(xp[i], r2), wp[k][i]), silu);
           }
           if (valid)
-            *reinterpret_cast<uint4*>(a.y + grow * N + c * 8) = pairs_to_bf16x8(yp);
+            *reinterpret_cast<uint4*>(a.y + grow * a.ldy + c * 8) = pairs_to_bf16x8(yp);
         }
       }
     }

@@ -13,7 +13,7 @@ constexpr int kMaxStages = 16;       // mbarrier pairs reserved in the shared-me
 constexpr int kHeaderBytes = 1024;   // barriers, block ids, flags and reduction slots
 constexpr int kRedSlotOffset = 512;  // float slots for cross-warp row reductions
 constexpr int kWorkspaceHeader = 256;  // workspace bytes before the dw partials
-constexpr int kReduceThreads = 512;  // dw second pass: 16 partial lanes x 32 column quads
+constexpr int kReduceThreads = 1024;  // dw second pass: 32 partial lanes x 32 column quads
 
 // Computing threads per CTA for a row geometry: 8 warps, or one 16-warp row group for the
 // widest rows.  One more warp (the producer) issues the copies.
@@ -28,6 +28,12 @@ GNORM_HD constexpr int max_ctas_per_sm(int kind, int threads_per_row, int chunks
   return threads_per_row > 256 ? 1
          : kind == 0            ? (chunks_per_thread == 1 ? 3 : (chunks_per_thread <= 4 ? 2 : 1))
                                 : (chunks_per_thread == 1 ? 2 : 1);
+}
+
+// Bytes one tensor of a pipeline stage occupies: R rows of N BF16 values, rounded up to
+// 128 bytes so every tensor of a stage starts 128-byte aligned (as tiled TMA copies require).
+GNORM_HD constexpr long long stage_tensor_bytes(long long rows, long long n) {
+  return (rows * n * 2 + 127) / 128 * 128;
 }
 
 }  // namespace gnorm

@@ -124,6 +124,8 @@ extern "C" int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, c
   a.rstd = rstd;
   a.dx = static_cast<uint16_t*>(dx);
   a.dg = static_cast<uint16_t*>(dg);
+  a.lddy = a.ldx = a.ldg = a.lddx = a.lddg = N;  // packed rows, BF16 weight
+  a.w_fp32 = 0;
   a.partial = reinterpret_cast<float*>(sc.ptr + kWorkspaceHeader);
   a.dw = dw;
   a.work_counter = reinterpret_cast<unsigned long long*>(sc.ptr);

@@ -120,7 +120,8 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   }
 
   // A stage holds R rows of each tensor; the backward's also holds their R FP32 rstd values.
-  const int64_t stage_raw = static_cast<int64_t>(tensors) * R * N * 2 + (kind == 1 ? R * 4 : 0);
+  const int64_t stage_raw = static_cast<int64_t>(tensors) * stage_tensor_bytes(R, N) +
+                            (kind == 1 ? R * 4 : 0);
   const int64_t stage_bytes = (stage_raw + 127) / 128 * 128;
   int64_t stages = std::min<int64_t>(max_stages, budget / stage_bytes);
   if (stages < 2) return GNORM_ERR_UNSUPPORTED;

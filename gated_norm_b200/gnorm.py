@@ -12,7 +12,7 @@ import threading
 
 import torch
 
-from ._lib import GNORM_OK, GnormPlan, GnormTuning, lib
+from ._lib import GNORM_OK, GnormBwdDesc, GnormFwdDesc, GnormPlan, GnormTuning, lib
 
 __all__ = [
     "GnormError",
@@ -26,6 +26,7 @@ __all__ = [
     "gnorm_status_string",
     "gnorm_plan_query",
     "gnorm_device_error",
+    "gnorm_selftest_wait_timeout",
     "gnorm_set_tuning",
     "gnorm_build_info",
     "workspace",
@@ -70,6 +71,14 @@ def gnorm_device_error(reset: bool = False) -> int:
     return int(lib.gnorm_device_error(int(bool(reset))))
 
 
+def gnorm_selftest_wait_timeout(timeout_us: int = 20000) -> int:
+    """Make one bounded wait run out on purpose; returns how long it waited (ns)."""
+    waited = ctypes.c_ulonglong(0)
+    _check(lib.gnorm_selftest_wait_timeout(int(timeout_us), ctypes.byref(waited)),
+           "gnorm_selftest_wait_timeout")
+    return int(waited.value)
+
+
 def gnorm_set_tuning(**knobs) -> None:
     """Process-wide experiment knobs (fields of gnorm_tuning; 0 = built-in).  No arguments
     restores every built-in choice.  Tri-state knobs (l2_prefetch, tail_reduce,
@@ -95,17 +104,25 @@ def _stream(stream, device) -> ctypes.c_void_p:
     return ctypes.c_void_p(stream.cuda_stream)
 
 
-def _rows(t: torch.Tensor, name: str):
+def _mat(t: torch.Tensor, name: str):
+    """(M, N, row stride) of a BF16 CUDA tensor viewed as rows of its last dimension.
+
+    Contiguous tensors of any rank are rows of the last dimension; a 2-D view with unit
+    column stride may have any row stride (e.g. a column slice of a wider buffer)."""
     if t.dim() < 1:
         raise ValueError(f"{name} must have a last dimension N")
     if t.dtype != torch.bfloat16:
         raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
-    if not t.is_contiguous():
-        raise ValueError(f"{name} must be contiguous (packed rows)")
     if t.device.type != "cuda":
         raise ValueError(f"{name} must be a CUDA tensor")
     N = t.shape[-1]
-    return t.numel() // N if N else 0, N
+    if t.is_contiguous():
+        return (t.numel() // N if N else 0), N, N
+    if t.dim() == 2 and t.stride(1) == 1:
+        M = t.shape[0]
+        return M, N, (t.stride(0) if M > 1 else N)
+    raise ValueError(f"{name}: rows need unit column stride (2-D row-strided views or "
+                     "contiguous tensors)")
 
 
 def _same(a: torch.Tensor, b: torch.Tensor, an: str, bn: str):
@@ -120,6 +137,11 @@ def _vec(t: torch.Tensor, N: int, dtypes, name: str, device):
         raise TypeError(f"{name} must be one of {dtypes}, got {t.dtype}")
     if t.numel() != N or not t.is_contiguous() or t.device != device:
         raise ValueError(f"{name} must be a contiguous [{N}] tensor on {device}")
+
+
+def _weight(w, N, device):
+    _vec(w, N, (torch.bfloat16, torch.float32), "w", device)
+    return 1 if w.dtype == torch.float32 else 0
 
 
 def _check(st: int, where: str):
@@ -151,64 +173,95 @@ def workspace(M: int, N: int, deterministic: bool, device) -> torch.Tensor:
 
 # ------------------------------------------------------------------------- entry points
 
-def gnorm_fwd(x, g, w, eps: float = 1e-6, *, y=None, rstd=None, stream=None):
-    """Forward: returns (y, rstd).  x, g: [..., N] BF16; w: [N] BF16; rstd: FP32 [M]."""
-    M, N = _rows(x, "x")
-    _rows(g, "g")
+def _fwd_desc(x, g, w, eps, y, rstd):
+    M, N, ldx = _mat(x, "x")
+    Mg, Ng, ldg = _mat(g, "g")
     _same(x, g, "x", "g")
-    _vec(w, N, (torch.bfloat16,), "w", x.device)
+    w_fp32 = _weight(w, N, x.device)
     if y is None:
-        y = torch.empty_like(x)
+        y = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
     else:
-        _rows(y, "y")
         _same(x, y, "x", "y")
+    _, _, ldy = _mat(y, "y")
     if rstd is None:
         rstd = torch.empty(M, dtype=torch.float32, device=x.device)
     else:
         _vec(rstd, M, (torch.float32,), "rstd", x.device)
-    with torch.cuda.device(x.device):
-        st = lib.gnorm_fwd(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(y), _ptr(rstd), M, N,
-                           _stream(stream, x.device))
-    _check(st, "gnorm_fwd")
-    return y, rstd
+    d = GnormFwdDesc(x=_ptr(x), ldx=ldx, g=_ptr(g), ldg=ldg, w=_ptr(w), w_fp32=w_fp32,
+                     eps=float(eps), y=_ptr(y), ldy=ldy, rstd=_ptr(rstd), M=M, N=N)
+    return d, y, rstd
 
 
-def _bwd_outputs(x, N, dx, dg, dw, dw_fp32):
+def _bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic, ws):
+    M, N, ldx = _mat(x, "x")
+    _, _, lddy = _mat(dy, "dy")
+    _, _, ldg = _mat(g, "g")
+    _same(x, dy, "x", "dy")
+    _same(x, g, "x", "g")
+    w_fp32 = _weight(w, N, x.device)
+    if rstd is not None:
+        _vec(rstd, M, (torch.float32,), "rstd", x.device)
     if dx is None:
-        dx = torch.empty_like(x)
-    else:
-        _rows(dx, "dx")
-        _same(x, dx, "x", "dx")
+        dx = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
     if dg is None:
-        dg = torch.empty_like(x)
-    else:
-        _rows(dg, "dg")
-        _same(x, dg, "x", "dg")
+        dg = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    _same(x, dx, "x", "dx")
+    _same(x, dg, "x", "dg")
+    _, _, lddx = _mat(dx, "dx")
+    _, _, lddg = _mat(dg, "dg")
     dw_dtype = torch.float32 if dw_fp32 else torch.bfloat16
     if dw is None:
         dw = torch.empty(N, dtype=dw_dtype, device=x.device)
     else:
         _vec(dw, N, (dw_dtype,), "dw", x.device)
-    return dx, dg, dw
+    if ws is None:
+        ws = workspace(M, N, deterministic, x.device)
+    d = GnormBwdDesc(dy=_ptr(dy), lddy=lddy, x=_ptr(x), ldx=ldx, g=_ptr(g), ldg=ldg, w=_ptr(w),
+                     w_fp32=w_fp32, rstd=_ptr(rstd), dx=_ptr(dx), lddx=lddx, dg=_ptr(dg),
+                     lddg=lddg, dw=_ptr(dw), dw_fp32=int(bool(dw_fp32)),
+                     deterministic=int(bool(deterministic)), M=M, N=N, workspace=_ptr(ws),
+                     workspace_bytes=ws.numel() * ws.element_size())
+    return d, dx, dg, dw
+
+
+def gnorm_fwd(x, g, w, eps: float = 1e-6, *, y=None, rstd=None, stream=None):
+    """Forward: returns (y, rstd).
+
+    x, g: BF16 rows (contiguous, or 2-D views with any row stride); w: BF16 or FP32 [N];
+    rstd: FP32 [M].  y is allocated packed unless given (it may be a strided view)."""
+    d, y, rstd = _fwd_desc(x, g, w, eps, y, rstd)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_fwd_ex(ctypes.byref(d), _stream(stream, x.device))
+    _check(st, "gnorm_fwd")
+    return y, rstd
 
 
 def gnorm_bwd(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: bool = False,
               deterministic: bool = True, workspace_buf=None, stream=None):
-    """Backward: returns (dx, dg, dw).  dw is FP32 if dw_fp32 else BF16."""
-    M, N = _rows(x, "x")
-    for t, n in ((dy, "dy"), (g, "g")):
-        _rows(t, n)
-        _same(x, t, "x", n)
-    _vec(w, N, (torch.bfloat16,), "w", x.device)
-    _vec(rstd, M, (torch.float32,), "rstd", x.device)
-    dx, dg, dw = _bwd_outputs(x, N, dx, dg, dw, dw_fp32)
-    ws = workspace_buf if workspace_buf is not None else workspace(M, N, deterministic, x.device)
+    """Backward: returns (dx, dg, dw).  dw is FP32 if dw_fp32 else BF16.  Row-strided 2-D
+    views are accepted for dy, x, g, dx, dg; w may be BF16 or FP32."""
+    d, dx, dg, dw = _bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic,
+                              workspace_buf)
+    if rstd is None:
+        raise ValueError("rstd is required")
     with torch.cuda.device(x.device):
-        st = lib.gnorm_bwd(_ptr(dy), _ptr(x), _ptr(g), _ptr(w), _ptr(rstd), _ptr(dx), _ptr(dg),
-                           _ptr(dw), int(bool(dw_fp32)), int(bool(deterministic)), M, N, _ptr(ws),
-                           ws.numel() * ws.element_size(), _stream(stream, x.device))
+        st = lib.gnorm_bwd_ex(ctypes.byref(d), _stream(stream, x.device))
     _check(st, "gnorm_bwd")
     return dx, dg, dw
+
+
+def gnorm_ckpt_step(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=None, dw=None,
+                    dw_fp32: bool = False, deterministic: bool = True, workspace_buf=None,
+                    stream=None):
+    """Checkpointed step (forward, forward again, backward): returns (y, rstd, dx, dg, dw)."""
+    fd, y, rstd = _fwd_desc(x, g, w, eps, y, rstd)
+    bd, dx, dg, dw = _bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic,
+                               workspace_buf)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_ckpt_step_ex(ctypes.byref(fd), ctypes.byref(bd),
+                                    _stream(stream, x.device))
+    _check(st, "gnorm_ckpt_step")
+    return y, rstd, dx, dg, dw
 
 
 def gnorm_dw_reduce(partials, *, dw=None, dw_fp32: bool = True, stream=None):
@@ -235,42 +288,26 @@ def gnorm_bwd_noalloc(dy, x, g, w, rstd, *, dx=None, dg=None, dw=None, dw_fp32: 
     For callers that cannot allocate device memory.  Calls that overlap on the GPU share
     the scratch and race; see include/gnorm.h.
     """
-    M, N = _rows(x, "x")
+    M, N, _ = _mat(x, "x")
     for t, n in ((dy, "dy"), (g, "g")):
-        _rows(t, n)
         _same(x, t, "x", n)
+    if dx is None:
+        dx = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    if dg is None:
+        dg = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    for t, n in ((x, "x"), (dy, "dy"), (g, "g"), (dx, "dx"), (dg, "dg")):
+        if _mat(t, n)[2] != N:
+            raise ValueError(f"gnorm_bwd_noalloc takes packed rows only ({n} is strided)")
     _vec(w, N, (torch.bfloat16,), "w", x.device)
     _vec(rstd, M, (torch.float32,), "rstd", x.device)
-    dx, dg, dw = _bwd_outputs(x, N, dx, dg, dw, dw_fp32)
+    dw_dtype = torch.float32 if dw_fp32 else torch.bfloat16
+    if dw is None:
+        dw = torch.empty(N, dtype=dw_dtype, device=x.device)
+    else:
+        _vec(dw, N, (dw_dtype,), "dw", x.device)
     with torch.cuda.device(x.device):
         st = lib.gnorm_bwd_noalloc(_ptr(dy), _ptr(x), _ptr(g), _ptr(w), _ptr(rstd), _ptr(dx),
                                    _ptr(dg), _ptr(dw), int(bool(dw_fp32)),
                                    int(bool(deterministic)), M, N, _stream(stream, x.device))
     _check(st, "gnorm_bwd_noalloc")
     return dx, dg, dw
-
-
-def gnorm_ckpt_step(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=None, dw=None,
-                    dw_fp32: bool = False, deterministic: bool = True, workspace_buf=None,
-                    stream=None):
-    """Checkpointed step (forward, forward again, backward): returns (y, rstd, dx, dg, dw)."""
-    M, N = _rows(x, "x")
-    for t, n in ((dy, "dy"), (g, "g")):
-        _rows(t, n)
-        _same(x, t, "x", n)
-    _vec(w, N, (torch.bfloat16,), "w", x.device)
-    if y is None:
-        y = torch.empty_like(x)
-    if rstd is None:
-        rstd = torch.empty(M, dtype=torch.float32, device=x.device)
-    else:
-        _vec(rstd, M, (torch.float32,), "rstd", x.device)
-    dx, dg, dw = _bwd_outputs(x, N, dx, dg, dw, dw_fp32)
-    ws = workspace_buf if workspace_buf is not None else workspace(M, N, deterministic, x.device)
-    with torch.cuda.device(x.device):
-        st = lib.gnorm_ckpt_step(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(dy), _ptr(y),
-                                 _ptr(rstd), _ptr(dx), _ptr(dg), _ptr(dw), int(bool(dw_fp32)),
-                                 int(bool(deterministic)), M, N, _ptr(ws),
-                                 ws.numel() * ws.element_size(), _stream(stream, x.device))
-    _check(st, "gnorm_ckpt_step")
-    return y, rstd, dx, dg, dw

@@ -122,6 +122,68 @@ GNORM_API int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, co
                                 int deterministic, int64_t M, int64_t N, void* stream);
 
 /*
+ * Strided rows and an FP32 weight.  Flashinfer PR #8701's commit message specialises its
+ * forward for inputs "where x and z hold their rows packed", so its API also takes rows
+ * that are not packed; these descriptors carry a row stride per tensor.  ld* = elements
+ * between the starts of consecutive rows (0 means N, i.e. packed); a stride must be >= N
+ * and a multiple of 8 (rows start 16-byte aligned).  w is FP32 [N] if w_fp32 != 0, else
+ * BF16.  rstd and dw are always packed vectors.  Outputs may share a buffer with other
+ * tensors as long as no element is shared (e.g. dx and dg as the two column halves of one
+ * [M, 2N] gradient): the alias check is exact for tensors with the same stride and
+ * conservative (whole byte extents) otherwise.  All other rules are those of gnorm_fwd /
+ * gnorm_bwd; the packed entry points are these with every stride N and a BF16 weight.
+ */
+typedef struct gnorm_fwd_desc {
+  const void* x;
+  int64_t ldx;
+  const void* g;
+  int64_t ldg;
+  const void* w;
+  int w_fp32;
+  float eps;
+  void* y;
+  int64_t ldy;
+  float* rstd;
+  int64_t M;
+  int64_t N;
+} gnorm_fwd_desc;
+
+typedef struct gnorm_bwd_desc {
+  const void* dy;
+  int64_t lddy;
+  const void* x;
+  int64_t ldx;
+  const void* g;
+  int64_t ldg;
+  const void* w;
+  int w_fp32;
+  const float* rstd;
+  void* dx;
+  int64_t lddx;
+  void* dg;
+  int64_t lddg;
+  void* dw;
+  int dw_fp32;
+  int deterministic;
+  int64_t M;
+  int64_t N;
+  void* workspace;
+  size_t workspace_bytes;
+} gnorm_bwd_desc;
+
+GNORM_API int gnorm_fwd_ex(const gnorm_fwd_desc* desc, void* stream);
+GNORM_API int gnorm_bwd_ex(const gnorm_bwd_desc* desc, void* stream);
+
+/*
+ * Checkpointed step with descriptors: x, g, w, eps, y, rstd, M, N come from `fwd`; dy, dx,
+ * dg, dw, dw_fp32, deterministic and the workspace from `bwd`, whose x, g, w, rstd fields
+ * must be NULL or equal to the forward's (same pointers, strides and weight type), and whose
+ * M and N must equal the forward's.
+ */
+GNORM_API int gnorm_ckpt_step_ex(const gnorm_fwd_desc* fwd, const gnorm_bwd_desc* bwd,
+                                 void* stream);
+
+/*
  * Checkpointed training step: forward, forward again (activation recomputation), backward,
  * all enqueued on `stream`.  Flashinfer PR #8701, section "How the tables were measured":
  * "ckptg" is the checkpointed step (2 x forward + backward), "stepg_f32" the same with an
@@ -189,7 +251,8 @@ GNORM_API int gnorm_plan_query(int kind, int64_t M, int64_t N, int deterministic
 
 /*
  * Device-side error word: kernels set a bit here if a bounded wait inside them gave up
- * (1 = a wait for copied data, 2 = a wait for a free pipeline stage).  Synchronises the
+ * (1 = a wait for copied data, 2 = a wait for a free pipeline stage, 4 = the self-test's
+ * wait, see gnorm_selftest_wait_timeout).  Synchronises the
  * current device, returns the word and clears it if `reset` != 0.  Returns -1 (as an int)
  * if the word cannot be read.
  */
@@ -213,6 +276,16 @@ typedef struct gnorm_tuning {
 } gnorm_tuning;
 
 GNORM_API void gnorm_set_tuning(const gnorm_tuning* tuning);
+
+/*
+ * Self-test of the bounded waits every kernel uses: launches one thread that waits on a
+ * barrier nothing arrives on, with a limit of `timeout_us` microseconds (1 .. 1000000).
+ * The wait gives up, sets bit 4 in the device error word (see gnorm_device_error) and the
+ * kernel returns; no fault, trap or hang.  Writes the time the wait took before giving up
+ * to *waited_ns (0 would mean the wait completed, which it cannot).  Synchronises the
+ * device and allocates 8 bytes: a diagnostic, not for use inside graphs.
+ */
+GNORM_API int gnorm_selftest_wait_timeout(unsigned timeout_us, unsigned long long* waited_ns);
 
 /* Build description: compiler version, target architecture (static storage). */
 GNORM_API const char* gnorm_build_info(void);

@@ -10,6 +10,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import gated_norm_b200 as gn
 from gated_norm_b200._lib import (GNORM_ERR_ARG, GNORM_ERR_NULL, GNORM_ERR_SHAPE, LIB_PATH,
@@ -65,6 +66,9 @@ def test_host_checks_precede_cuda():
         GNORM_ERR_NULL
     assert lib.gnorm_ckpt_step(p, p, p, 1e-6, p, p, p, p, p, p, 0, 1, 4, 7, p, 1 << 20, None) == \
         GNORM_ERR_SHAPE
+    waited = ctypes.c_ulonglong(0)
+    assert lib.gnorm_selftest_wait_timeout(0, ctypes.byref(waited)) == GNORM_ERR_ARG
+    assert lib.gnorm_selftest_wait_timeout(1000, None) == GNORM_ERR_NULL
 
 
 # ------------------------------------------------------------------------- dispatch rule
@@ -89,7 +93,8 @@ def test_plan_invariants(sms, kind):
                 assert p["consumer_threads"] % p["threads_per_row"] == 0
                 assert p["consumer_threads"] + 32 <= 1024
                 tensors = 2 if kind == 0 else 3
-                stage = -(-(tensors * R * N * 2 + (4 * R if kind == 1 else 0)) // 128) * 128
+                tensor = -(-(R * N * 2) // 128) * 128
+                stage = -(-(tensors * tensor + (4 * R if kind == 1 else 0)) // 128) * 128
                 assert p["smem_bytes"] >= 1024 + p["stages"] * stage
                 assert p["smem_bytes"] <= 232448
                 # static round-robin: no CTA gets more than one block above the mean
@@ -228,3 +233,49 @@ def test_tail_and_l2_knobs_in_plans():
     finally:
         gn.gnorm_set_tuning()
     assert gn.gnorm_plan_query(1, 65536, 128, True, 148) == base
+
+
+# ------------------------------------------------------------ strided rows (host checks)
+
+def _fwd_desc(**kw):
+    from gated_norm_b200._lib import GnormFwdDesc
+    base = dict(x=1 << 20, ldx=0, g=2 << 20, ldg=0, w=3 << 20, w_fp32=0, eps=1e-6,
+                y=4 << 20, ldy=0, rstd=5 << 20, M=4, N=128)
+    base.update(kw)
+    return GnormFwdDesc(**base)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="fake pointers that pass the host checks would reach a launch")
+def test_strided_descriptor_checks_precede_cuda():
+    """Stride and alias rules are host checks; a descriptor that passes them goes on to the
+    device query, which fails without a GPU (GNORM_ERR_CUDA), so the two are told apart."""
+    from gated_norm_b200._lib import (GNORM_ERR_ALIAS, GNORM_ERR_ALIGN, GNORM_ERR_CUDA,
+                                      GNORM_ERR_SHAPE)
+    fwd = lambda **kw: lib.gnorm_fwd_ex(ctypes.byref(_fwd_desc(**kw)), None)
+    assert fwd(ldx=100) == GNORM_ERR_SHAPE            # stride shorter than a row
+    assert fwd(ldx=132) == GNORM_ERR_ALIGN            # rows would not start 16-byte aligned
+    base = 1 << 24
+    # x and g as the two column halves of one [M, 256] buffer (inputs may share memory)
+    assert fwd(x=base, ldx=256, g=base + 256, ldg=256) == GNORM_ERR_CUDA
+    # y in the other half of x's buffer: no element shared -> passes the alias check
+    assert fwd(x=base, ldx=256, y=base + 256, ldy=256) == GNORM_ERR_CUDA
+    # y shifted by 8 columns into x's rows: shares elements -> rejected
+    assert fwd(x=base, ldx=256, y=base + 16, ldy=256) == GNORM_ERR_ALIAS
+    # y one whole row below x with the same stride: rows overlap -> rejected
+    assert fwd(x=base, ldx=256, y=base + 512, ldy=256) == GNORM_ERR_ALIAS
+    # y past the end of x's last row
+    assert fwd(x=base, ldx=256, y=base + 4 * 512, ldy=256) == GNORM_ERR_CUDA
+    # different strides that interleave: the check is conservative -> rejected
+    assert fwd(x=base, ldx=256, y=base + 256, ldy=384) == GNORM_ERR_ALIAS
+
+
+def test_ckpt_ex_requires_consistent_descriptors():
+    from gated_norm_b200._lib import GNORM_ERR_ARG, GnormBwdDesc
+    f = _fwd_desc()
+    b = GnormBwdDesc(dy=6 << 20, x=7 << 20, dx=8 << 20, dg=9 << 20, dw=10 << 20, M=4, N=128,
+                     workspace=11 << 20, workspace_bytes=1 << 20)
+    assert lib.gnorm_ckpt_step_ex(ctypes.byref(f), ctypes.byref(b), None) == GNORM_ERR_ARG
+    b.x = f.x
+    b.M = 5
+    assert lib.gnorm_ckpt_step_ex(ctypes.byref(f), ctypes.byref(b), None) == GNORM_ERR_ARG
