@@ -393,7 +393,7 @@ def run_ours(args, wl):
     bwd_traffic = profiled_traffic("bwd_kernel", wl.name)
     achieved = gbs["bwd"]
     cpu = None
-    if not args.no_cpu_baseline:
+    if not args.no_cpu_baseline and world == 1:  # the CPU baseline runs at N = 1 only
         c_gbs, c_rows, c_reps, c_sec = time_oracle(wl, args.cpu_seconds)
         cpu = {"value": c_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"{c_rows} of {wl.M} rows x N={N}, {c_reps} checkpointed steps "

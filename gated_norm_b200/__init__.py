@@ -4,6 +4,7 @@ The kernels live in ``libgnorm.so`` behind the C ABI of ``include/gnorm.h``; thi
 is a thin binding over it.  Importing the package loads the library and fails loudly if it
 has not been built (``python gated_norm_b200/build.py``): there is no CPU fallback.
 """
+from .autograd import GatedRMSNorm, GatedRMSNormFunction, gated_rmsnorm  # noqa: F401
 from .gnorm import (  # noqa: F401
     GnormError,
     gnorm_build_info,

@@ -279,3 +279,20 @@ def test_ckpt_ex_requires_consistent_descriptors():
     b.x = f.x
     b.M = 5
     assert lib.gnorm_ckpt_step_ex(ctypes.byref(f), ctypes.byref(b), None) == GNORM_ERR_ARG
+
+
+def test_header_is_c_and_links_from_c(tmp_path):
+    """include/gnorm.h compiles as C99 and a C program links and calls libgnorm."""
+    exe = tmp_path / "c_abi_example"
+    libdir = os.path.dirname(LIB_PATH)
+    src = os.path.join(ROOT, "tests", "c_abi_example.c")
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    src, "-o", str(exe), "-L", libdir, "-lgnorm", f"-Wl,-rpath,{libdir}"],
+                   check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    fields = dict(kv.split("=") for kv in out.split()[:7])
+    p = gn.gnorm_plan_query(1, 368640, 128, True, 148)
+    assert int(fields["grid"]) == p["grid"] and int(fields["rows"]) == p["rows_per_stage"]
+    assert int(fields["ws"]) == gn.gnorm_bwd_workspace_bytes_for(368640, 128, True, 148)
+    assert int(fields["null"]) == GNORM_ERR_NULL and int(fields["shape"]) == GNORM_ERR_SHAPE
+    assert "sm_100a" in out
