@@ -4,14 +4,21 @@
 
 namespace gnorm {
 
+template <int TPR, int CPT, bool kWFp32>
+static cudaError_t launch_bwd_weight(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream,
+                                      bool pdl) {
+  const void* k = reinterpret_cast<const void*>(&gated_rmsnorm_bwd_kernel<TPR, CPT, kWFp32>);
+  cudaError_t e = ensure_smem_limit(k, p.smem_bytes);
+  if (e != cudaSuccess) return e;
+  return launch_kernel(gated_rmsnorm_bwd_kernel<TPR, CPT, kWFp32>, p.grid,
+                       consumer_threads_for(TPR) + 32, p.smem_bytes, stream, pdl, a);
+}
+
 template <int TPR, int CPT>
 static cudaError_t launch_bwd_geometry(const gnorm_plan& p, const BwdArgs& a,
                                        cudaStream_t stream, bool pdl) {
-  const void* k = reinterpret_cast<const void*>(&gated_rmsnorm_bwd_kernel<TPR, CPT>);
-  cudaError_t e = ensure_smem_limit(k, p.smem_bytes);
-  if (e != cudaSuccess) return e;
-  return launch_kernel(gated_rmsnorm_bwd_kernel<TPR, CPT>, p.grid, consumer_threads_for(TPR) + 32,
-                       p.smem_bytes, stream, pdl, a);
+  return a.w_fp32 ? launch_bwd_weight<TPR, CPT, true>(p, a, stream, pdl)
+                  : launch_bwd_weight<TPR, CPT, false>(p, a, stream, pdl);
 }
 
 cudaError_t launch_bwd(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream, bool pdl) {

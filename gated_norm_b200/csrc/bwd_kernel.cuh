@@ -117,7 +117,7 @@ __global__ void __launch_bounds__(kReduceThreads)
   if (work_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0ull;
 }
 
-template <int TPR, int CPT>
+template <int TPR, int CPT, bool kWFp32>
 __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(1, TPR, CPT))
     gated_rmsnorm_bwd_kernel(const __grid_constant__ BwdArgs a) {
   constexpr int kNCT = consumer_threads_for(TPR);
@@ -272,7 +272,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
       wp[k][i] = splat2(0.f);
       dwacc[k][i] = splat2(0.f);
     }
-    if (cval[k]) load_weight_pairs(a.w, a.w_fp32, c, wp[k]);
+    if (cval[k]) load_weight_pairs<kWFp32>(a.w, c, wp[k]);
   }
 
   int s = 0;

@@ -262,9 +262,12 @@ __device__ __forceinline__ void copy_row_block(uint8_t* dst, const uint16_t* src
   }
 }
 
-// This thread's 8 weights of chunk c as FP32 pairs, from a BF16 or FP32 weight vector.
-__device__ __forceinline__ void load_weight_pairs(const void* w, int w_fp32, int c, float2 p[4]) {
-  if (w_fp32) {
+// This thread's 8 weights of chunk c as FP32 pairs, from a BF16 or (kWFp32) FP32 weight
+// vector.  The weight type is a compile-time choice: a runtime branch here measurably slowed
+// the wide-row backward.
+template <bool kWFp32>
+__device__ __forceinline__ void load_weight_pairs(const void* w, int c, float2 p[4]) {
+  if constexpr (kWFp32) {
     const float4* w4 = reinterpret_cast<const float4*>(w) + 2 * c;
     const float4 a = w4[0], b = w4[1];
     p[0] = make_float2(a.x, a.y);

@@ -22,7 +22,7 @@
 namespace gnorm {
 
 
-template <int TPR, int CPT>
+template <int TPR, int CPT, bool kWFp32>
 __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(0, TPR, CPT))
     gated_rmsnorm_fwd_kernel(const __grid_constant__ FwdArgs a) {
   constexpr int kNCT = consumer_threads_for(TPR);
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_s
     cval[k] = c < n8;
 #pragma unroll
     for (int i = 0; i < 4; ++i) wp[k][i] = splat2(0.f);
-    if (cval[k]) load_weight_pairs(a.w, a.w_fp32, c, wp[k]);
+    if (cval[k]) load_weight_pairs<kWFp32>(a.w, c, wp[k]);
   }
 
   int s = 0;
