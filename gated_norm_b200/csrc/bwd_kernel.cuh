@@ -118,9 +118,9 @@ __global__ void __launch_bounds__(kReduceThreads)
 }
 
 template <int TPR, int CPT, bool kWFp32>
-__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(1, TPR, CPT))
+__global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ctas_per_sm(1, TPR, CPT))
     gated_rmsnorm_bwd_kernel(const __grid_constant__ BwdArgs a) {
-  constexpr int kNCT = consumer_threads_for(TPR);
+  constexpr int kNCT = consumer_threads_for(1, TPR, CPT);
   constexpr int kGroups = kNCT / TPR;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);

@@ -11,7 +11,7 @@ static cudaError_t launch_fwd_weight(const gnorm_plan& p, const FwdArgs& a, cuda
   cudaError_t e = ensure_smem_limit(k, p.smem_bytes);
   if (e != cudaSuccess) return e;
   return launch_kernel(gated_rmsnorm_fwd_kernel<TPR, CPT, kWFp32>, p.grid,
-                       consumer_threads_for(TPR) + 32, p.smem_bytes, stream, pdl, a);
+                       consumer_threads_for(0, TPR, CPT) + 32, p.smem_bytes, stream, pdl, a);
 }
 
 template <int TPR, int CPT>

@@ -23,9 +23,9 @@ namespace gnorm {
 
 
 template <int TPR, int CPT, bool kWFp32>
-__global__ void __launch_bounds__(consumer_threads_for(TPR) + 32, max_ctas_per_sm(0, TPR, CPT))
+__global__ void __launch_bounds__(consumer_threads_for(0, TPR, CPT) + 32, max_ctas_per_sm(0, TPR, CPT))
     gated_rmsnorm_fwd_kernel(const __grid_constant__ FwdArgs a) {
-  constexpr int kNCT = consumer_threads_for(TPR);
+  constexpr int kNCT = consumer_threads_for(0, TPR, CPT);
   constexpr int kGroups = kNCT / TPR;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);

@@ -15,19 +15,23 @@ constexpr int kRedSlotOffset = 512;  // float slots for cross-warp row reduction
 constexpr int kWorkspaceHeader = 256;  // workspace bytes before the dw partials
 constexpr int kReduceThreads = 1024;  // dw second pass: 32 partial lanes x 32 column quads
 
-// Computing threads per CTA for a row geometry: 8 warps, or one 16-warp row group for the
-// widest rows.  One more warp (the producer) issues the copies.
-GNORM_HD constexpr int consumer_threads_for(int threads_per_row) {
-  return threads_per_row > 256 ? threads_per_row : 256;
+// Computing threads per CTA for a row geometry: 8 warps; one 16-warp row group for the
+// widest rows; and 16 warps for the backward of narrow rows (<= 16 threads per row, one
+// chunk per thread), which is latency-bound with 8 (measured on B200: the 368640 x 128
+// checkpointed step 181 -> 176 us).  One more warp (the producer) issues the copies.
+GNORM_HD constexpr int consumer_threads_for(int kind, int threads_per_row, int chunks_per_thread) {
+  return threads_per_row > 256 ? threads_per_row
+         : (kind == 1 && threads_per_row <= 16 && chunks_per_thread == 1) ? 512
+                                                                           : 256;
 }
 
 // Resident CTAs per SM a kernel is compiled for (its __launch_bounds__ minimum), which caps
 // its registers: 3 CTAs of 288 threads leave 75 registers per thread, 2 leave 113.  The
 // dispatch rule never plans more CTAs per SM than this.
 GNORM_HD constexpr int max_ctas_per_sm(int kind, int threads_per_row, int chunks_per_thread) {
-  return threads_per_row > 256 ? 1
-         : kind == 0            ? (chunks_per_thread == 1 ? 3 : (chunks_per_thread <= 4 ? 2 : 1))
-                                : (chunks_per_thread == 1 ? 2 : 1);
+  return consumer_threads_for(kind, threads_per_row, chunks_per_thread) > 256 ? 1
+         : kind == 0 ? (chunks_per_thread == 1 ? 3 : (chunks_per_thread <= 4 ? 2 : 1))
+                     : (chunks_per_thread == 1 ? 2 : 1);
 }
 
 // Bytes one tensor of a pipeline stage occupies: R rows of N BF16 values, rounded up to

@@ -71,7 +71,7 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
         static_cast<int64_t>(geo.threads_per_row) * geo.chunks_per_thread * 8 < N)
       return GNORM_ERR_UNSUPPORTED;
   }
-  const int nct = consumer_threads_for(geo.threads_per_row);
+  const int nct = consumer_threads_for(kind, geo.threads_per_row, geo.chunks_per_thread);
   const int groups = nct / geo.threads_per_row;
   const int tensors = kind == 0 ? 2 : 3;
   const int64_t row_bytes = static_cast<int64_t>(tensors) * N * 2;

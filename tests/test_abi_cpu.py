@@ -92,6 +92,8 @@ def test_plan_invariants(sms, kind):
                 assert p["threads_per_row"] * p["chunks_per_thread"] * 8 >= N
                 assert p["consumer_threads"] % p["threads_per_row"] == 0
                 assert p["consumer_threads"] + 32 <= 1024
+                if kind == 1 and p["threads_per_row"] <= 16 and p["chunks_per_thread"] == 1:
+                    assert p["consumer_threads"] == 512
                 tensors = 2 if kind == 0 else 3
                 tensor = -(-(R * N * 2) // 128) * 128
                 stage = -(-(tensors * tensor + (4 * R if kind == 1 else 0)) // 128) * 128
@@ -163,7 +165,7 @@ def test_ctas_per_sm_never_exceeds_the_compiled_residency():
                     finally:
                         gn.gnorm_set_tuning()
                     tpr, cpt = p["threads_per_row"], p["chunks_per_thread"]
-                    fit = 1 if tpr > 256 else (
+                    fit = 1 if p["consumer_threads"] > 256 else (
                         (3 if cpt == 1 else 2 if cpt <= 4 else 1) if kind == 0 else
                         (2 if cpt == 1 else 1))
                     assert p["ctas_per_sm"] <= fit
