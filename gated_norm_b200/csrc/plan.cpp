@@ -8,7 +8,8 @@
 // tier, and splits the rows evenly over the persistent CTAs:
 //   forward with < 512 KB of staged rows per SM : 3 CTAs per SM, ~16 KB stages (latency tier);
 //   other forwards                              : 2 CTAs per SM, ~48 KB stages;
-//   backward                                    : 1 CTA per SM, ~48 KB (>= 3-row) stages;
+//   backward                                    : 1 CTA per SM, <= 3 stages of ~48 KB
+//                                                 (at least 3 rows);
 // and within a tier: if the rows per CTA fit in one stage, one block per CTA; otherwise k
 // equal blocks per CTA, block size chosen so all CTAs get the same number of rows.
 #include <algorithm>
@@ -86,8 +87,9 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   const int ctas_per_sm =
       std::min(fit, g_knobs.ctas_per_sm > 0 ? g_knobs.ctas_per_sm : default_ctas);
   const int64_t stage_target = g_knobs.stage_bytes > 0 ? g_knobs.stage_bytes : default_stage;
-  const int max_stages =
-      std::min(kMaxStages, g_knobs.max_stages > 0 ? g_knobs.max_stages : kMaxStages);
+  const int max_stages = std::min(
+      kMaxStages, g_knobs.max_stages > 0 ? g_knobs.max_stages
+                                         : (kind == 1 ? kBwdMaxStages : kMaxStages));
 
   // Shared memory available to one CTA when `ctas_per_sm` share an SM.
   int64_t smem_cta = smem_per_block;

@@ -23,6 +23,9 @@ constexpr int64_t kFwdLatencyStageBytes = 16384;
 constexpr int64_t kFwdLatencyTierBytes = 512 * 1024;
 constexpr int64_t kBwdStageBytes = 49152;
 constexpr int kBwdMinStageRows = 3;
+// At most 3 backward stages in flight per SM: measured best or equal on every workload
+// (368640x128 backward 89.2 -> 83.1 us with 3 instead of 4 stages of ~48 KB).
+constexpr int kBwdMaxStages = 3;
 // Measured on B200 in same-box A/B runs (graph replays, cold L2):
 //  * an L2 bulk prefetch of the block after each CTA's ring slows every workload (e.g.
 //    368640x128 forward 55 -> 68 us, backward 86 -> 113 us): off;
