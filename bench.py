@@ -7,7 +7,8 @@ A step is one checkpointed training step over one batch of seeded synthetic rows
 forward, forward again (recompute), backward with the dw reduction -- every stage of the
 path -- replayed from one CUDA graph ("ckptg").  Each timed step also replays the backward
 ("bwdg") and the forward ("fwdg") alone, each from its own graph, for the per-operation
-times and the roofline of the dominant kernel.  The default workload is 65536 x 128 (a
+times and the roofline of the dominant kernel (the forward: two launches per step, the
+largest share of the step's device time).  The default workload is 65536 x 128 (a
 per-head gated norm of a linear-attention output, 512 heads x 128 tokens).  Times are
 CUDA-event device times on the launching stream; L2 is flushed (256 MiB write) before
 every timed replay, outside the events.  `value` is the checkpointed step's algorithmic
@@ -15,7 +16,10 @@ HBM bytes of the whole job / the max-over-ranks summed step time (GB/s).
 
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the
 data path; the rows of a data-parallel batch are independent).  `--impl reference` times
-the FP64 CPU oracle on a bounded sample of the same workload (rank 0 only).
+the FP64 CPU oracle on a bounded sample of the same workload (rank 0 only).  `--floor`
+adds, after the timed region, the same measurement of an empty graph and of torch
+elementwise kernels that move the forward's and backward's main streams (context for the
+fixed per-launch cost at small sizes).
 """
 from __future__ import annotations
 
@@ -245,6 +249,48 @@ def run_reference(args, wl):
 
 # ----------------------------------------------------------------------------- our leg
 
+def measure_floor(torch, dev, stream, flush, x, g, dy, y, dx, K):
+    """The timing method's own floor: an empty graph (one one-element add) and torch
+    elementwise kernels over the same [M, N] BF16 tensors -- y = x * g (the forward's
+    reads and write) and dx = x + g * dy (three reads, one write) -- each replayed from a
+    CUDA graph between the same L2 flush and events as the timed steps."""
+    one = torch.zeros(1, device=dev)
+    ops = {
+        "empty_graph": (0, lambda: one.add_(1)),
+        "torch_mul": (3 * x.numel() * 2, lambda: torch.mul(x, g, out=y)),
+        "torch_addcmul": (4 * x.numel() * 2, lambda: torch.addcmul(x, g, dy, out=dx)),
+    }
+    reps = max(20, min(K, 200))
+    out = {}
+    for name, (nbytes, fn) in ops.items():
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+            fn()
+        stream.wait_stream(side)
+        torch.cuda.synchronize(dev)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            fn()
+        for _ in range(3):
+            flush.zero_()
+            graph.replay()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(reps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        t_us = statistics.mean(a.elapsed_time(b) * 1e3 for a, b in evs)
+        out[name] = {"us": t_us, "bytes": nbytes,
+                     "gbs": (nbytes / (t_us * 1e-6) / 1e9) if nbytes else None}
+        del graph
+    return out
+
+
 def run_ours(args, wl):
     import torch
 
@@ -377,6 +423,8 @@ def run_ours(args, wl):
                "path": "gnorm_ckpt_step with pinned host inputs copied in and outputs copied "
                        "back on the same stream each step"}
 
+    floor = measure_floor(torch, dev, stream, flush, x, g, dy, y, dx, K) if args.floor else None
+
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -390,8 +438,12 @@ def run_ours(args, wl):
     gbs = {"fwd": fwd_bytes(M, N) / (us["fwd"] * 1e-6) / 1e9,
            "bwd": bwd_bytes(M, N, fp32) / (us["bwd"] * 1e-6) / 1e9,
            "ckpt": step_bytes / (us["ckpt"] * 1e-6) / 1e9}
+    fwd_traffic = profiled_traffic("fwd_kernel", wl.name)
     bwd_traffic = profiled_traffic("bwd_kernel", wl.name)
-    achieved = gbs["bwd"]
+    # device time of one step by kernel, from the standalone replays: the forward kernel
+    # (twice) and the backward operation (kernel + second pass)
+    step_us = 2 * us["fwd"] + us["bwd"]
+    shares = {"fwd_kernel_x2": 2 * us["fwd"] / step_us, "bwd_op": us["bwd"] / step_us}
     cpu = None
     if not args.no_cpu_baseline and world == 1:  # the CPU baseline runs at N = 1 only
         c_gbs, c_rows, c_reps, c_sec = time_oracle(wl, args.cpu_seconds)
@@ -411,17 +463,27 @@ def run_ours(args, wl):
         "timing": "fwd, bwd, ckpt each replayed from its own CUDA graph (fwdg, bwdg, ckptg)",
         "gbs": gbs,
         "frac_of_peak": {k: v / peak for k, v in gbs.items()},
-        "roofline": {"bound": "hbm", "kernel": "gnorm_bwd (backward kernel + dw second pass, "
-                                                "graph-replayed)",
-                     "achieved": achieved, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": achieved / peak,
-                     "algorithmic_bytes_per_launch": bwd_bytes(M, N, fp32),
-                     "traffic": bwd_traffic},
+        "roofline": {"bound": "hbm",
+                     "kernel": "gated_rmsnorm_fwd_kernel (one launch per fwdg replay)",
+                     "achieved": gbs["fwd"], "peak": peak, "peak_kind": peak_kind,
+                     "unit": "GB/s", "frac": gbs["fwd"] / peak,
+                     "algorithmic_bytes_per_launch": fwd_bytes(M, N),
+                     "traffic": fwd_traffic},
+        "roofline_bwd": {"bound": "hbm",
+                         "kernel": "gnorm_bwd (backward kernel + dw second pass, one bwdg "
+                                   "replay)",
+                         "achieved": gbs["bwd"], "peak": peak, "peak_kind": peak_kind,
+                         "unit": "GB/s", "frac": gbs["bwd"] / peak,
+                         "algorithmic_bytes_per_launch": bwd_bytes(M, N, fp32),
+                         "traffic": bwd_traffic},
+        "step_shares": shares,
         "cpu_baseline": cpu,
         "e2e": e2e,
         "gpu_launches": sum(launches.values()) * K,
         "clocks": clk,
     }
+    if floor is not None:
+        line["floor"] = floor
     print(json.dumps(line))
     return 0
 
@@ -438,6 +500,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--floor", action="store_true",
+                    help="also time an empty graph and torch elementwise kernels the same way")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="target duration of the reference (oracle) arm")
     args = ap.parse_args(argv)

@@ -29,7 +29,7 @@ KNOB_SETS = [
 ]
 
 
-@pytest.mark.parametrize("M,N", [(4099, 128), (700, 4096), (2500, 256)])
+@pytest.mark.parametrize("M,N", [(4099, 128), (700, 4096), (2500, 256), (1337, 40), (777, 16)])
 @pytest.mark.parametrize("det", [True, False])
 def test_knobs_do_not_change_results(M, N, det):
     case = Case(M, N, seed=23)
