@@ -395,17 +395,17 @@ def run_ours(args, wl):
     e2e = None
     if args.e2e_steps > 0:
         hx, hg, hdy, hw = (t.cpu().pin_memory() for t in (x, g, dy, w))
-        outs_h = [torch.empty_like(t, device="cpu").pin_memory() for t in (y, rstd, dx, dg, dw)]
+        hy, hr, hdx, hdg, hdw = (torch.empty_like(t, device="cpu").pin_memory()
+                                 for t in (y, rstd, dx, dg, dw))
         h2d = sum(t.numel() * t.element_size() for t in (hx, hg, hdy, hw))
-        d2h = sum(t.numel() * t.element_size() for t in outs_h)
+        d2h = sum(t.numel() * t.element_size() for t in (hy, hr, hdx, hdg, hdw))
+        dev_buf = torch.empty(gn.gnorm_ckpt_step_host_bytes(M, N, det), dtype=torch.uint8,
+                              device=dev)
 
         def e2e_step():
-            for h, dv in zip((hx, hg, hdy, hw), (x, g, dy, w)):
-                dv.copy_(h, non_blocking=True)
-            gn.gnorm_ckpt_step(x, g, w, eps, dy, y=y, rstd=rstd, dx=dx, dg=dg, dw=dw,
-                               dw_fp32=fp32, deterministic=det, workspace_buf=ws, stream=stream)
-            for h, dv in zip(outs_h, (y, rstd, dx, dg, dw)):
-                h.copy_(dv, non_blocking=True)
+            gn.gnorm_ckpt_step_host(hx, hg, hw, eps, hdy, y=hy, rstd=hr, dx=hdx, dg=hdg, dw=hdw,
+                                    dw_fp32=fp32, deterministic=det, dev_buf=dev_buf,
+                                    device=dev, stream=stream)
 
         for _ in range(3):
             e2e_step()
@@ -420,8 +420,9 @@ def run_ours(args, wl):
         e2e = {"value": whole_job_gbs(step_bytes, args.e2e_steps, world, e_ms), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "ms_per_step": e_ms / args.e2e_steps,
-               "path": "gnorm_ckpt_step with pinned host inputs copied in and outputs copied "
-                       "back on the same stream each step"}
+               "path": "gnorm_ckpt_step_host: pinned host inputs and outputs; the library "
+                       "copies each step's inputs in and outputs back, chunk by chunk, "
+                       "overlapping both directions of the host link with the kernels"}
 
     floor = measure_floor(torch, dev, stream, flush, x, g, dy, y, dx, K) if args.floor else None
 

@@ -13,6 +13,8 @@ from .gnorm import (  # noqa: F401
     gnorm_bwd_workspace_bytes,
     gnorm_bwd_workspace_bytes_for,
     gnorm_ckpt_step,
+    gnorm_ckpt_step_host,
+    gnorm_ckpt_step_host_bytes,
     gnorm_device_error,
     gnorm_dw_reduce,
     gnorm_fwd,

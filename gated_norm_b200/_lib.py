@@ -52,7 +52,8 @@ class GnormTuning(ctypes.Structure):
 
     _fields_ = [(name, ctypes.c_int) for name in (
         "stage_bytes", "max_stages", "ctas_per_sm", "disable_pdl", "threads_per_row",
-        "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch")]
+        "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch",
+        "host_chunk_bytes")]
 
 
 class GnormFwdDesc(ctypes.Structure):
@@ -105,6 +106,9 @@ SIGNATURES = {
     "gnorm_ckpt_step_ex": (_int, [ctypes.POINTER(GnormFwdDesc), ctypes.POINTER(GnormBwdDesc), _vp]),
     "gnorm_ckpt_step": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
                                _i64, _vp, _sz, _vp]),
+    "gnorm_ckpt_step_host": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int,
+                                    _int, _i64, _i64, _vp, _sz, _vp]),
+    "gnorm_ckpt_step_host_bytes": (_sz, [_i64, _i64, _int]),
     "gnorm_dw_reduce": (_int, [_vp, _i64, _i64, _vp, _int, _vp]),
     "gnorm_bwd_workspace_bytes": (_sz, [_i64, _i64, _int]),
     "gnorm_bwd_workspace_bytes_for": (_sz, [_i64, _i64, _int, _int]),

@@ -28,7 +28,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libgnorm.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "plan.cpp", "noalloc.cu"]
+SOURCES = ["api.cu", "fwd.cu", "bwd.cu", "plan.cpp", "noalloc.cu", "host_step.cu"]
 
 
 def nvcc() -> str:

@@ -574,6 +574,7 @@ void gnorm_set_tuning(const gnorm_tuning* tuning) {
     k.l2_prefetch = tri(k.l2_prefetch);
     k.tail_reduce = tri(k.tail_reduce);
     k.chain_prefetch = tri(k.chain_prefetch);
+    k.host_chunk_bytes = clamp0(k.host_chunk_bytes);
   }
   set_tuning(k);
 }

@@ -19,6 +19,8 @@ __all__ = [
     "gnorm_fwd",
     "gnorm_bwd",
     "gnorm_ckpt_step",
+    "gnorm_ckpt_step_host",
+    "gnorm_ckpt_step_host_bytes",
     "gnorm_bwd_noalloc",
     "gnorm_dw_reduce",
     "gnorm_bwd_workspace_bytes",
@@ -261,6 +263,61 @@ def gnorm_ckpt_step(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=N
         st = lib.gnorm_ckpt_step_ex(ctypes.byref(fd), ctypes.byref(bd),
                                     _stream(stream, x.device))
     _check(st, "gnorm_ckpt_step")
+    return y, rstd, dx, dg, dw
+
+
+def gnorm_ckpt_step_host_bytes(M: int, N: int, deterministic: bool = True) -> int:
+    return int(lib.gnorm_ckpt_step_host_bytes(int(M), int(N), int(bool(deterministic))))
+
+
+def _host_mat(t, M, N, name):
+    if t.device.type != "cpu" or t.dtype != torch.bfloat16 or not t.is_contiguous() or \
+            tuple(t.shape) != (M, N):
+        raise ValueError(f"{name} must be a contiguous BF16 [{M}, {N}] CPU tensor")
+
+
+def gnorm_ckpt_step_host(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=None,
+                         dw=None, dw_fp32: bool = False, deterministic: bool = True,
+                         dev_buf=None, device=None, stream=None):
+    """Checkpointed step on HOST tensors (pinned for overlapped copies): the library copies
+    the rows in, runs the step chunk by chunk and copies the outputs back, all ordered on
+    `stream` of `device`.  Returns (y, rstd, dx, dg, dw) as CPU tensors; they are written
+    once the stream has reached the end of the call."""
+    if x.dim() != 2:
+        raise ValueError("x must be a 2-D [M, N] CPU tensor")
+    M, N = x.shape
+    for t, n in ((x, "x"), (g, "g"), (dy, "dy")):
+        _host_mat(t, M, N, n)
+    if w.device.type != "cpu" or w.dtype != torch.bfloat16 or tuple(w.shape) != (N,):
+        raise ValueError(f"w must be a BF16 [{N}] CPU tensor")
+    pin = x.is_pinned()
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None \
+        else torch.device(device)
+
+    def new(shape, dtype):
+        return torch.empty(shape, dtype=dtype, pin_memory=pin)
+
+    y = new((M, N), torch.bfloat16) if y is None else y
+    dx = new((M, N), torch.bfloat16) if dx is None else dx
+    dg = new((M, N), torch.bfloat16) if dg is None else dg
+    rstd = new((M,), torch.float32) if rstd is None else rstd
+    dw_dtype = torch.float32 if dw_fp32 else torch.bfloat16
+    dw = new((N,), dw_dtype) if dw is None else dw
+    for t, n in ((y, "y"), (dx, "dx"), (dg, "dg")):
+        _host_mat(t, M, N, n)
+    for t, n, length, dt in ((rstd, "rstd", M, torch.float32), (dw, "dw", N, dw_dtype)):
+        if t.device.type != "cpu" or t.dtype != dt or tuple(t.shape) != (length,):
+            raise ValueError(f"{n} must be a {dt} [{length}] CPU tensor")
+    with torch.cuda.device(device):
+        need = gnorm_ckpt_step_host_bytes(M, N, deterministic)
+        if dev_buf is None:
+            dev_buf = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+        st = lib.gnorm_ckpt_step_host(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(dy), _ptr(y),
+                                      _ptr(rstd), _ptr(dx), _ptr(dg), _ptr(dw),
+                                      int(bool(dw_fp32)), int(bool(deterministic)), M, N,
+                                      _ptr(dev_buf), dev_buf.numel() * dev_buf.element_size(),
+                                      _stream(stream, device))
+    _check(st, "gnorm_ckpt_step_host")
     return y, rstd, dx, dg, dw
 
 

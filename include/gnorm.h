@@ -196,6 +196,43 @@ GNORM_API int gnorm_ckpt_step(const void* x, const void* g, const void* w, float
                     void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Checkpointed step on HOST buffers (no counterpart in the pages: an entry point for callers
+ * whose batch lives in host memory).  x, g, dy [M, N] BF16 and w [N] BF16 are read from host
+ * memory; y, dx, dg [M, N] BF16, rstd [M] FP32 and dw [N] (FP32 if dw_fp32, else BF16) are
+ * written to host memory; all rows packed.  The rows are processed in chunks (about 4 MiB of
+ * x, g and dy each) as a pipeline over the caller's stream and two copy streams the library
+ * creates once per device: chunk k's inputs are copied in while chunk k-1's step runs and
+ * earlier chunks' outputs are copied out, so both directions of the host link work at once.
+ * Each chunk runs gnorm_ckpt_step with an FP32 dw of its own rows; dw is the fixed-order sum
+ * of those rows (gnorm_dw_reduce).  y, rstd, dx and dg are bitwise equal to gnorm_ckpt_step's;
+ * dw is too when there is one chunk (M x N x 6 bytes <= 4 MiB), and otherwise is rounded
+ * differently but is still bitwise stable run to run in deterministic mode.
+ *
+ * dev_buf: device scratch of at least gnorm_ckpt_step_host_bytes(M, N, deterministic) bytes,
+ *   GNORM_WORKSPACE_ALIGN-aligned, owned by the caller; it holds device copies of every
+ *   tensor, so it must not be shared by calls that may overlap on the GPU.  No state is kept
+ *   between calls.
+ * Host buffers: pinned memory (cudaHostAlloc / cudaHostRegister) makes the copies
+ *   asynchronous and lets them overlap; pageable memory works but serialises them and blocks
+ *   the calling thread.  Outputs may overlap neither an input nor each other
+ *   (GNORM_ERR_ALIAS).  The buffers must stay valid until `stream` has reached the end of
+ *   the call: it returns once everything is enqueued; the caller's stream waits for the
+ *   last copy out, so synchronising the stream (or an event recorded on it afterwards)
+ *   means every host output is written.  Errors: as gnorm_ckpt_step, and GNORM_ERR_WORKSPACE
+ *   for a missing, misaligned or small dev_buf.  Not meant for CUDA graph capture.
+ */
+GNORM_API int gnorm_ckpt_step_host(const void* x, const void* g, const void* w, float eps,
+                                   const void* dy, void* y, float* rstd, void* dx, void* dg,
+                                   void* dw, int dw_fp32, int deterministic, int64_t M, int64_t N,
+                                   void* dev_buf, size_t dev_bytes, void* stream);
+
+/*
+ * Device bytes gnorm_ckpt_step_host needs on the CURRENT device for this shape (0 if the
+ * arguments are invalid or no device is present).
+ */
+GNORM_API size_t gnorm_ckpt_step_host_bytes(int64_t M, int64_t N, int deterministic);
+
+/*
  * Fixed-order sum of P rows of FP32 partials [P, N] (device memory, row-major) into dw[N]
  * (BF16 if dw_fp32 == 0, else FP32), with the same kernel and summation order as the
  * backward's deterministic second pass (the fixed-order FP32 partial reduction of flashinfer
@@ -273,6 +310,7 @@ typedef struct gnorm_tuning {
   int l2_prefetch;       /* 1: warm L2 with the block after each CTA's ring, 2: do not */
   int tail_reduce;       /* 1: dw second pass in the backward's last CTA when small, 2: never */
   int chain_prefetch;    /* 1: in gnorm_ckpt_step, copy inputs before the previous kernel ends, 2: do not */
+  int host_chunk_bytes;  /* gnorm_ckpt_step_host: bytes of x, g and dy per chunk */
 } gnorm_tuning;
 
 GNORM_API void gnorm_set_tuning(const gnorm_tuning* tuning);
