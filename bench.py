@@ -207,6 +207,39 @@ def time_oracle(wl, min_seconds, max_rows=65536, seed=0):
     return gbs, rows, done, el
 
 
+def _oracle_worker(job):
+    """One spawned process: the oracle's checkpointed step on its own seeded row sample,
+    repeated until `seconds` have passed; returns (bytes done, seconds)."""
+    name, rows, seed, seconds = job
+    import oracle
+
+    wl = WORKLOADS[name]
+    d = make_inputs(rows, wl.N, seed=seed, g_std=wl.g_std, outlier_frac=wl.outlier_frac)
+    x, g, dy, w = (bf16_bits_to_f64(d[k]) for k in ("x", "g", "dy", "w"))
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.ckpt_step(x, g, w, wl.eps, dy)
+        done += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            return ckpt_bytes(rows, wl.N, True) * done, el
+
+
+def time_oracle_all_cores(wl, seconds, max_procs=64, rows_per_proc=8192):
+    """The same oracle on every usable host core at once (one spawned process per core,
+    each on its own row sample, as a row partition of the batch would run); returns
+    (aggregate GB/s, processes, rows per process)."""
+    import multiprocessing as mp
+
+    procs = max(1, min(len(os.sched_getaffinity(0)), max_procs))
+    rows = min(wl.M, rows_per_proc)
+    jobs = [(wl.name, rows, wl.seed + 1000 + i, seconds) for i in range(procs)]
+    with mp.get_context("spawn").Pool(procs) as pool:
+        res = pool.map(_oracle_worker, jobs)
+    gbs = sum(b / el for b, el in res) / 1e9
+    return gbs, procs, rows
+
+
 def run_reference(args, wl):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -424,6 +457,18 @@ def run_ours(args, wl):
                        "copies each step's inputs in and outputs back, chunk by chunk, "
                        "overlapping both directions of the host link with the kernels"}
 
+    # the forward launched eagerly (no graph), same flush and events, after the timed region
+    fwd_eager = []
+    for i in range(min(K, 200) + 3):
+        flush.zero_()
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a_ev.record(stream)
+        op_fwd()
+        b_ev.record(stream)
+        fwd_eager.append((a_ev, b_ev))
+    torch.cuda.synchronize(dev)
+    fwd_eager_us = statistics.mean(a_ev.elapsed_time(b_ev) for a_ev, b_ev in fwd_eager[3:]) * 1e3
+
     floor = measure_floor(torch, dev, stream, flush, x, g, dy, y, dx, K) if args.floor else None
 
     if world > 1:
@@ -436,6 +481,14 @@ def run_ours(args, wl):
         return float(sum(v) / len(v))
 
     us = {"fwd": avg(t_fwd) * 1e3, "bwd": avg(t_bwd) * 1e3, "ckpt": avg(t_ckpt) * 1e3}
+
+    def median_of_rounds(v, rounds=10):
+        n = max(1, len(v) // rounds)
+        meds = [statistics.median(v[i:i + n]) for i in range(0, n * (len(v) // n), n)]
+        return statistics.median(meds) * 1e3
+
+    us_median = {"fwd": median_of_rounds(t_fwd), "bwd": median_of_rounds(t_bwd),
+                 "ckpt": median_of_rounds(t_ckpt)}
     gbs = {"fwd": fwd_bytes(M, N) / (us["fwd"] * 1e-6) / 1e9,
            "bwd": bwd_bytes(M, N, fp32) / (us["bwd"] * 1e-6) / 1e9,
            "ckpt": step_bytes / (us["ckpt"] * 1e-6) / 1e9}
@@ -445,12 +498,18 @@ def run_ours(args, wl):
     # (twice) and the backward operation (kernel + second pass)
     step_us = 2 * us["fwd"] + us["bwd"]
     shares = {"fwd_kernel_x2": 2 * us["fwd"] / step_us, "bwd_op": us["bwd"] / step_us}
-    cpu = None
+    cpu = cpu_all = None
     if not args.no_cpu_baseline and world == 1:  # the CPU baseline runs at N = 1 only
         c_gbs, c_rows, c_reps, c_sec = time_oracle(wl, args.cpu_seconds)
         cpu = {"value": c_gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
                "sample": f"{c_rows} of {wl.M} rows x N={N}, {c_reps} checkpointed steps "
                          f"in {c_sec:.1f} s (FP64 numpy oracle, one core)"}
+        if args.cpu_all_cores:
+            a_gbs, a_procs, a_rows = time_oracle_all_cores(wl, args.cpu_seconds)
+            cpu_all = {"value": a_gbs, "unit": "GB/s", "cores": a_procs, "kind": "oracle",
+                       "sample": f"{a_procs} processes, each {a_rows} rows x N={N} of its own, "
+                                 f"checkpointed steps for {args.cpu_seconds:.0f} s "
+                                 "(FP64 numpy oracle, one process per core)"}
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
@@ -461,6 +520,8 @@ def run_ours(args, wl):
                    "l2": "flushed between steps (256 MiB write, outside the timed events)",
                    "parallelism": f"dp{world} (independent rows per rank, no collective)"},
         "us_per_call": us,
+        "us_median_of_round_medians": us_median,
+        "us_fwd_eager": fwd_eager_us,
         "timing": "fwd, bwd, ckpt each replayed from its own CUDA graph (fwdg, bwdg, ckptg)",
         "gbs": gbs,
         "frac_of_peak": {k: v / peak for k, v in gbs.items()},
@@ -479,6 +540,7 @@ def run_ours(args, wl):
                          "traffic": bwd_traffic},
         "step_shares": shares,
         "cpu_baseline": cpu,
+        "cpu_baseline_all_cores": cpu_all,
         "e2e": e2e,
         "gpu_launches": sum(launches.values()) * K,
         "clocks": clk,
@@ -501,6 +563,8 @@ def main(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-cpu-all-cores", dest="cpu_all_cores", action="store_false",
+                    help="skip the oracle timed on all host cores")
     ap.add_argument("--floor", action="store_true",
                     help="also time an empty graph and torch elementwise kernels the same way")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
