@@ -173,6 +173,23 @@ def workspace(M: int, N: int, deterministic: bool, device) -> torch.Tensor:
         return buf
 
 
+_host_cache: dict = {}
+
+
+def _host_step_buffer(M: int, N: int, deterministic: bool, device) -> torch.Tensor:
+    """Device buffer for gnorm_ckpt_step_host, cached per device and grown as needed (calls
+    that may overlap on the GPU must pass buffers of their own)."""
+    idx = device.index if device.index is not None else torch.cuda.current_device()
+    with torch.cuda.device(idx):
+        need = max(gnorm_ckpt_step_host_bytes(M, N, deterministic), 256)
+    with _ws_lock:
+        buf = _host_cache.get(idx)
+        if buf is None or buf.numel() < need:
+            buf = torch.empty(need, dtype=torch.uint8, device=torch.device("cuda", idx))
+            _host_cache[idx] = buf
+        return buf
+
+
 # ------------------------------------------------------------------------- entry points
 
 def _fwd_desc(x, g, w, eps, y, rstd):
@@ -309,9 +326,8 @@ def gnorm_ckpt_step_host(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None,
         if t.device.type != "cpu" or t.dtype != dt or tuple(t.shape) != (length,):
             raise ValueError(f"{n} must be a {dt} [{length}] CPU tensor")
     with torch.cuda.device(device):
-        need = gnorm_ckpt_step_host_bytes(M, N, deterministic)
         if dev_buf is None:
-            dev_buf = torch.empty(max(need, 256), dtype=torch.uint8, device=device)
+            dev_buf = _host_step_buffer(M, N, deterministic, device)
         st = lib.gnorm_ckpt_step_host(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(dy), _ptr(y),
                                       _ptr(rstd), _ptr(dx), _ptr(dg), _ptr(dw),
                                       int(bool(dw_fp32)), int(bool(deterministic)), M, N,
