@@ -110,10 +110,19 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+# Host code of entry points bench.py does not call (the kernels, and the code that plans
+# and launches them for bench.py, live in the other files): a change there leaves recorded
+# ncu counters valid.
+_DIGEST_EXCLUDED = ("host_step.cu", "noalloc.cu")
+
+
 def source_digest():
+    """Digest of the kernel sources and of the host code that plans and launches them."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_norm_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if name in _DIGEST_EXCLUDED:
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
