@@ -145,14 +145,13 @@ extern "C" int gnorm_ckpt_step_host(const void* x, const void* g, const void* w,
                                     const void* dy, void* y, float* rstd, void* dx, void* dg,
                                     void* dw, int dw_fp32, int deterministic, int64_t M,
                                     int64_t N, void* dev_buf, size_t dev_bytes, void* stream) {
-  HostLayout L;
-  int st = host_layout(M, N, deterministic, &L);
-  if (st != GNORM_OK) return st;
+  // Argument checks first, before any CUDA call.
+  if (M < 0 || N < 8 || N > GNORM_N_MAX || (N % 8) != 0 || M > (int64_t(1) << 40))
+    return GNORM_ERR_SHAPE;
   if (!std::isfinite(eps) || eps < 0.f) return GNORM_ERR_ARG;
   if (!dw) return GNORM_ERR_NULL;
   if (M > 0 && (!x || !g || !w || !dy || !y || !rstd || !dx || !dg)) return GNORM_ERR_NULL;
-  if (!dev_buf || reinterpret_cast<uintptr_t>(dev_buf) % GNORM_WORKSPACE_ALIGN != 0 ||
-      dev_bytes < L.total)
+  if (!dev_buf || reinterpret_cast<uintptr_t>(dev_buf) % GNORM_WORKSPACE_ALIGN != 0)
     return GNORM_ERR_WORKSPACE;
   // Host outputs may overlap neither a host input nor each other.
   const size_t mat = static_cast<size_t>(M) * N * 2;
@@ -167,6 +166,10 @@ extern "C" int gnorm_ckpt_step_host(const void* x, const void* g, const void* w,
     for (int j = i + 1; j < 5; ++j)
       if (spans_overlap(out_p[i], out_n[i], out_p[j], out_n[j])) return GNORM_ERR_ALIAS;
   }
+  HostLayout L;
+  int st = host_layout(M, N, deterministic, &L);  // queries the device
+  if (st != GNORM_OK) return st;
+  if (dev_bytes < L.total) return GNORM_ERR_WORKSPACE;
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return GNORM_ERR_CUDA;

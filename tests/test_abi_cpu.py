@@ -272,6 +272,36 @@ def test_strided_descriptor_checks_precede_cuda():
     assert fwd(x=base, ldx=256, y=base + 256, ldy=384) == GNORM_ERR_ALIAS
 
 
+@pytest.mark.skipif(torch.cuda.is_available(),
+                    reason="fake pointers that pass the host checks would reach a copy")
+def test_host_step_checks_precede_cuda():
+    """gnorm_ckpt_step_host checks its arguments before any CUDA call; arguments that pass
+    go on to the device query, which fails without a GPU (GNORM_ERR_CUDA)."""
+    from gated_norm_b200._lib import GNORM_ERR_ALIAS, GNORM_ERR_CUDA, GNORM_ERR_WORKSPACE
+
+    def call(M=64, N=128, eps=1e-6, dev_buf=1 << 30, **ptrs):
+        p = {k: (i + 1) << 26 for i, k in enumerate(("x", "g", "w", "dy", "y", "rstd", "dx",
+                                                     "dg", "dw"))}
+        p.update(ptrs)
+        v = {k: ctypes.c_void_p(a) if a is not None else None for k, a in p.items()}
+        return lib.gnorm_ckpt_step_host(v["x"], v["g"], v["w"], eps, v["dy"], v["y"], v["rstd"],
+                                        v["dx"], v["dg"], v["dw"], 1, 1, M, N,
+                                        ctypes.c_void_p(dev_buf) if dev_buf else None, 1 << 30,
+                                        None)
+    assert call(N=12) == GNORM_ERR_SHAPE
+    assert call(M=-1) == GNORM_ERR_SHAPE
+    assert call(eps=float("inf")) == GNORM_ERR_ARG
+    assert call(dw=None) == GNORM_ERR_NULL
+    assert call(dg=None) == GNORM_ERR_NULL
+    assert call(dev_buf=None) == GNORM_ERR_WORKSPACE
+    assert call(dev_buf=(1 << 30) + 16) == GNORM_ERR_WORKSPACE  # not 256-byte aligned
+    assert call(y=(1 << 26) + 64) == GNORM_ERR_ALIAS            # y inside x
+    assert call(dx=(5 << 26) + 4096) == GNORM_ERR_ALIAS         # dx inside y
+    assert call() == GNORM_ERR_CUDA                             # passes: device query fails
+    assert lib.gnorm_ckpt_step_host_bytes(64, 128, 1) == 0      # no device
+    assert lib.gnorm_ckpt_step_host_bytes(64, 12, 1) == 0       # bad shape
+
+
 def test_ckpt_ex_requires_consistent_descriptors():
     from gated_norm_b200._lib import GNORM_ERR_ARG, GnormBwdDesc
     f = _fwd_desc()
