@@ -41,6 +41,7 @@ class GnormPlan(ctypes.Structure):
         ("fused_reduce", ctypes.c_int),
         ("partials", ctypes.c_int),
         ("l2_prefetch", ctypes.c_int),
+        ("direct_loads", ctypes.c_int),
     ]
 
     def as_dict(self) -> dict:
@@ -53,7 +54,7 @@ class GnormTuning(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int) for name in (
         "stage_bytes", "max_stages", "ctas_per_sm", "disable_pdl", "threads_per_row",
         "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch",
-        "host_chunk_bytes")]
+        "host_chunk_bytes", "fwd_direct")]
 
 
 class GnormFwdDesc(ctypes.Structure):

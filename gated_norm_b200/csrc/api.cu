@@ -206,8 +206,8 @@ int enqueue_fwd(const DeviceInfo& d, const gnorm_fwd_desc& f, cudaStream_t strea
   a.l2_prefetch = plan.l2_prefetch;
   a.err = d.err_word;
   const int R = plan.rows_per_stage;
-  if (rows_map(&a.map_x, f.x, f.M, f.N, f.ldx, R)) a.map_bits |= 1;
-  if (rows_map(&a.map_g, f.g, f.M, f.N, f.ldg, R)) a.map_bits |= 2;
+  if (!plan.direct_loads && rows_map(&a.map_x, f.x, f.M, f.N, f.ldx, R)) a.map_bits |= 1;
+  if (!plan.direct_loads && rows_map(&a.map_g, f.g, f.M, f.N, f.ldg, R)) a.map_bits |= 2;
   if (launch_fwd(plan, a, stream, use_pdl()) != cudaSuccess) return GNORM_ERR_CUDA;
   return GNORM_OK;
 }
@@ -575,6 +575,7 @@ void gnorm_set_tuning(const gnorm_tuning* tuning) {
     k.tail_reduce = tri(k.tail_reduce);
     k.chain_prefetch = tri(k.chain_prefetch);
     k.host_chunk_bytes = clamp0(k.host_chunk_bytes);
+    k.fwd_direct = tri(k.fwd_direct);
   }
   set_tuning(k);
 }

@@ -1,4 +1,5 @@
 // fwd.cu -- instantiations and launcher of the forward kernel.
+#include "fwd_direct.cuh"
 #include "fwd_kernel.cuh"
 #include "launch.h"
 
@@ -21,7 +22,27 @@ static cudaError_t launch_fwd_geometry(const gnorm_plan& p, const FwdArgs& a,
                   : launch_fwd_weight<TPR, CPT, false>(p, a, stream, pdl);
 }
 
+template <int TPR>
+static cudaError_t launch_fwd_direct(const gnorm_plan& p, const FwdArgs& a, cudaStream_t stream,
+                                     bool pdl) {
+  if (a.w_fp32)
+    return launch_kernel(gated_rmsnorm_fwd_direct_kernel<TPR, true>, p.grid, kDirectThreads, 0,
+                         stream, pdl, a);
+  return launch_kernel(gated_rmsnorm_fwd_direct_kernel<TPR, false>, p.grid, kDirectThreads, 0,
+                       stream, pdl, a);
+}
+
 cudaError_t launch_fwd(const gnorm_plan& p, const FwdArgs& a, cudaStream_t stream, bool pdl) {
+  if (p.direct_loads) {
+    if (p.chunks_per_thread != 1) return cudaErrorInvalidConfiguration;
+    switch (p.threads_per_row) {
+      case 4: return launch_fwd_direct<4>(p, a, stream, pdl);
+      case 8: return launch_fwd_direct<8>(p, a, stream, pdl);
+      case 16: return launch_fwd_direct<16>(p, a, stream, pdl);
+      case 32: return launch_fwd_direct<32>(p, a, stream, pdl);
+      default: return cudaErrorInvalidConfiguration;
+    }
+  }
   const int key = p.threads_per_row * 8 + p.chunks_per_thread;
   switch (key) {
     case 4 * 8 + 1: return launch_fwd_geometry<4, 1>(p, a, stream, pdl);

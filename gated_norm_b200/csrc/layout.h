@@ -34,6 +34,14 @@ GNORM_HD constexpr int max_ctas_per_sm(int kind, int threads_per_row, int chunks
                      : (chunks_per_thread == 1 ? 2 : 1);
 }
 
+// The forward for narrow rows in the latency tier loads its rows straight into registers
+// (gated_rmsnorm_fwd_direct_kernel): 256 threads per CTA, all computing; each row group
+// takes kDirectRows rows per iteration; kDirectCtasPerSm CTAs per SM (its
+// __launch_bounds__ minimum: 64 registers per thread).
+constexpr int kDirectThreads = 256;
+constexpr int kDirectRows = 2;
+constexpr int kDirectCtasPerSm = 4;
+
 // Bytes one tensor of a pipeline stage occupies: R rows of N BF16 values, rounded up to
 // 128 bytes so every tensor of a stage starts 128-byte aligned (as tiled TMA copies require).
 GNORM_HD constexpr long long stage_tensor_bytes(long long rows, long long n) {

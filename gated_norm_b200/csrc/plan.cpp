@@ -11,7 +11,9 @@
 //   backward                                    : 1 CTA per SM, <= 3 stages of ~48 KB
 //                                                 (at least 3 rows);
 // and within a tier: if the rows per CTA fit in one stage, one block per CTA; otherwise k
-// equal blocks per CTA, block size chosen so all CTAs get the same number of rows.
+// equal blocks per CTA, block size chosen so all CTAs get the same number of rows.  In the
+// forward's latency tier, rows of N <= 256 skip the staging altogether: 4 CTAs of 256
+// threads per SM load them straight into registers (gated_rmsnorm_fwd_direct_kernel).
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -80,6 +82,31 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   // Rows-per-SM tiers (bytes of staged rows per SM decide, so wide and narrow rows compare).
   const int64_t rows_per_sm = (M + num_sms - 1) / num_sms;
   const bool latency_tier = kind == 0 && rows_per_sm * row_bytes < kFwdLatencyTierBytes;
+  // Forward of narrow rows in the latency tier (or always / never, by knob): rows loaded
+  // straight into registers, no shared-memory stages.
+  const bool direct_capable = kind == 0 && geo.chunks_per_thread == 1 && geo.threads_per_row <= 32;
+  const bool direct = direct_capable && (g_knobs.fwd_direct == 1 ||
+                                         (g_knobs.fwd_direct == 0 && latency_tier));
+  if (direct) {
+    const int64_t rows_per_iter =
+        static_cast<int64_t>(kDirectThreads / geo.threads_per_row) * kDirectRows;
+    const int ctas = std::min(kDirectCtasPerSm,
+                              g_knobs.ctas_per_sm > 0 ? g_knobs.ctas_per_sm : kDirectCtasPerSm);
+    const int64_t blocks = ceil_div(M, rows_per_iter);
+    out->kind = 0;
+    out->threads_per_row = geo.threads_per_row;
+    out->chunks_per_thread = 1;
+    out->consumer_threads = kDirectThreads;
+    out->rows_per_stage = static_cast<int>(rows_per_iter);
+    out->stages = 0;
+    out->ctas_per_sm = ctas;
+    out->grid = static_cast<int>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * ctas));
+    out->num_blocks = blocks;
+    out->smem_bytes = 0;
+    out->direct_loads = 1;
+    return GNORM_OK;
+  }
+
   const int fit = max_ctas_per_sm(kind, geo.threads_per_row, geo.chunks_per_thread);
   const int default_ctas = kind == 1 ? 1 : (latency_tier ? 3 : 2);
   int64_t default_stage = kind == 1 ? std::max<int64_t>(kBwdStageBytes, kBwdMinStageRows * (row_bytes + 4))

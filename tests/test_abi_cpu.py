@@ -86,6 +86,17 @@ def test_plan_invariants(sms, kind):
             for det in (True, False):
                 p = gn.gnorm_plan_query(kind, M, N, det, sms)
                 R, G = p["rows_per_stage"], p["grid"]
+                rows_per_sm = -(-M // sms)
+                latency = rows_per_sm * 4 * N < 512 * 1024
+                assert p["direct_loads"] == (kind == 0 and N <= 256 and latency)
+                if p["direct_loads"]:  # rows straight into registers, no stages
+                    tpr = p["threads_per_row"]
+                    assert p["chunks_per_thread"] == 1 and tpr * 8 >= N and tpr <= 32
+                    assert p["consumer_threads"] == 256 and R == (256 // tpr) * 2
+                    assert p["stages"] == 0 and p["smem_bytes"] == 0
+                    assert p["num_blocks"] * R >= M and (p["num_blocks"] - 1) * R < M
+                    assert 1 <= G <= min(p["num_blocks"], 4 * sms) and p["ctas_per_sm"] == 4
+                    continue
                 assert 1 <= R and p["stages"] >= 2
                 assert p["num_blocks"] * R >= M and (p["num_blocks"] - 1) * R < M
                 assert 1 <= G <= sms * p["ctas_per_sm"] and G <= p["num_blocks"]
@@ -127,31 +138,46 @@ def test_tier_edge_rows_per_sm():
         rows_edge = 512 * 1024 // (4 * N)  # rows per SM where the staged bytes reach 512 KB
         lat = gn.gnorm_plan_query(0, (rows_edge - 1) * sms, N, True, sms)
         stream = gn.gnorm_plan_query(0, rows_edge * sms, N, True, sms)
-        assert lat["ctas_per_sm"] == 3 and stream["ctas_per_sm"] == 2
-        assert lat["rows_per_stage"] * 4 * N <= 16384 < stream["rows_per_stage"] * 4 * N
+        # narrow rows in the latency tier: loaded straight into registers, 4 CTAs per SM
+        assert lat["direct_loads"] == 1 and lat["ctas_per_sm"] == 4 and lat["stages"] == 0
+        assert stream["direct_loads"] == 0 and stream["ctas_per_sm"] == 2
+        try:  # with staging forced, the latency tier stages ~16 KB with 3 CTAs per SM
+            gn.gnorm_set_tuning(fwd_direct=2)
+            lat = gn.gnorm_plan_query(0, (rows_edge - 1) * sms, N, True, sms)
+            assert lat["direct_loads"] == 0 and lat["ctas_per_sm"] == 3
+            assert lat["rows_per_stage"] * 4 * N <= 16384 < stream["rows_per_stage"] * 4 * N
+            gn.gnorm_set_tuning(fwd_direct=1)  # and loads straight into registers at any size
+            assert gn.gnorm_plan_query(0, rows_edge * sms, N, True, sms)["direct_loads"] == 1
+            assert gn.gnorm_plan_query(0, rows_edge * sms, 264, True, sms)["direct_loads"] == 0
+        finally:
+            gn.gnorm_set_tuning()
         # the wide-row forward uses the same byte rule; its registers cap it at 2 CTAs per SM
         wide_lat = gn.gnorm_plan_query(0, 8 * sms, 4096, True, sms)
         wide_stream = gn.gnorm_plan_query(0, 64 * sms, 4096, True, sms)
         assert wide_lat["ctas_per_sm"] == wide_stream["ctas_per_sm"] == 2
         assert wide_lat["rows_per_stage"] == 1 and wide_stream["rows_per_stage"] == 3
-        for kind in (0, 1):
-            big = gn.gnorm_plan_query(kind, 1 << 12, N, True, sms)
-            ctas = sms * big["ctas_per_sm"]
-            edge = None
-            for rows_per_cta in range(1, 400):
-                p = gn.gnorm_plan_query(kind, rows_per_cta * ctas, N, True, sms)
-                if p["ctas_per_sm"] != big["ctas_per_sm"]:
-                    break
-                if p["num_blocks"] > p["grid"]:
-                    edge = rows_per_cta
-                    break
-            if edge is None:
-                continue
-            below = gn.gnorm_plan_query(kind, (edge - 1) * ctas, N, True, sms)
-            above = gn.gnorm_plan_query(kind, edge * ctas, N, True, sms)
-            assert below["num_blocks"] == below["grid"] == ctas
-            assert below["rows_per_stage"] == edge - 1
-            assert above["num_blocks"] > above["grid"]
+        try:
+            gn.gnorm_set_tuning(fwd_direct=2)  # the staged forward's blocks
+            for kind in (0, 1):
+                big = gn.gnorm_plan_query(kind, 1 << 12, N, True, sms)
+                ctas = sms * big["ctas_per_sm"]
+                edge = None
+                for rows_per_cta in range(1, 400):
+                    p = gn.gnorm_plan_query(kind, rows_per_cta * ctas, N, True, sms)
+                    if p["ctas_per_sm"] != big["ctas_per_sm"]:
+                        break
+                    if p["num_blocks"] > p["grid"]:
+                        edge = rows_per_cta
+                        break
+                if edge is None:
+                    continue
+                below = gn.gnorm_plan_query(kind, (edge - 1) * ctas, N, True, sms)
+                above = gn.gnorm_plan_query(kind, edge * ctas, N, True, sms)
+                assert below["num_blocks"] == below["grid"] == ctas
+                assert below["rows_per_stage"] == edge - 1
+                assert above["num_blocks"] > above["grid"]
+        finally:
+            gn.gnorm_set_tuning()
 
 
 def test_ctas_per_sm_never_exceeds_the_compiled_residency():
@@ -168,6 +194,8 @@ def test_ctas_per_sm_never_exceeds_the_compiled_residency():
                     fit = 1 if p["consumer_threads"] > 256 else (
                         (3 if cpt == 1 else 2 if cpt <= 4 else 1) if kind == 0 else
                         (2 if cpt == 1 else 1))
+                    if p["direct_loads"]:
+                        fit = 4  # the direct-load forward's compiled residency
                     assert p["ctas_per_sm"] <= fit
 
 

@@ -26,6 +26,8 @@ KNOB_SETS = [
     dict(disable_pdl=1),
     dict(ctas_per_sm=1, stage_bytes=8192, max_stages=2),
     dict(ctas_per_sm=2, stage_bytes=98304),
+    dict(fwd_direct=1),
+    dict(fwd_direct=2),
 ]
 
 
@@ -53,4 +55,33 @@ def test_knobs_do_not_change_results(M, N, det):
                 assert rep["ok"], (knobs, rep)
     finally:
         gn.gnorm_set_tuning()
+    assert gn.gnorm_device_error(reset=True) == 0
+
+
+@pytest.mark.parametrize("M,N", [(1, 8), (37, 16), (1000, 40), (4099, 128), (2500, 256),
+                                 (70001, 128)])
+@pytest.mark.parametrize("w_fp32", [False, True])
+@pytest.mark.parametrize("strided", [False, True])
+def test_direct_and_staged_forward_agree(M, N, w_fp32, strided):
+    """The forward that loads rows straight into registers and the one that stages them in
+    shared memory do the same arithmetic in the same order: bitwise equal y and rstd, for
+    packed and strided rows (x and g as the column halves of one buffer) and both weight
+    types."""
+    case = Case(M, N, seed=29)
+    if strided:
+        xg = torch.cat([case.x, case.g], dim=1)
+        x, g = xg[:, :N], xg[:, N:]
+    else:
+        x, g = case.x, case.g
+    w = case.w.float() if w_fp32 else case.w
+    outs = []
+    try:
+        for mode in (1, 2):
+            gn.gnorm_set_tuning(fwd_direct=mode)
+            assert gn.gnorm_plan_query(0, M, N, True, 148)["direct_loads"] == (mode == 1)
+            outs.append(gn.gnorm_fwd(x, g, w, case.eps))
+        torch.cuda.synchronize()
+    finally:
+        gn.gnorm_set_tuning()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
     assert gn.gnorm_device_error(reset=True) == 0
