@@ -54,7 +54,7 @@ class GnormTuning(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int) for name in (
         "stage_bytes", "max_stages", "ctas_per_sm", "disable_pdl", "threads_per_row",
         "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch",
-        "host_chunk_bytes", "fwd_direct")]
+        "host_chunk_bytes", "fwd_direct", "bwd_direct")]
 
 
 class GnormFwdDesc(ctypes.Structure):

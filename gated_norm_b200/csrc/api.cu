@@ -249,9 +249,11 @@ int enqueue_bwd(const DeviceInfo& d, const gnorm_bwd_desc& b, cudaStream_t strea
   a.l2_prefetch = plan.l2_prefetch;
   a.err = d.err_word;
   const int R = plan.rows_per_stage;
-  if (rows_map(&a.map_dy, b.dy, b.M, b.N, b.lddy, R)) a.map_bits |= 1;
-  if (rows_map(&a.map_x, b.x, b.M, b.N, b.ldx, R)) a.map_bits |= 2;
-  if (rows_map(&a.map_g, b.g, b.M, b.N, b.ldg, R)) a.map_bits |= 4;
+  if (!plan.direct_loads) {
+    if (rows_map(&a.map_dy, b.dy, b.M, b.N, b.lddy, R)) a.map_bits |= 1;
+    if (rows_map(&a.map_x, b.x, b.M, b.N, b.ldx, R)) a.map_bits |= 2;
+    if (rows_map(&a.map_g, b.g, b.M, b.N, b.ldg, R)) a.map_bits |= 4;
+  }
   const bool pdl = use_pdl();
   if (launch_bwd(plan, a, stream, pdl) != cudaSuccess) return GNORM_ERR_CUDA;
   if (!plan.fused_reduce) {
@@ -576,6 +578,7 @@ void gnorm_set_tuning(const gnorm_tuning* tuning) {
     k.chain_prefetch = tri(k.chain_prefetch);
     k.host_chunk_bytes = clamp0(k.host_chunk_bytes);
     k.fwd_direct = tri(k.fwd_direct);
+    k.bwd_direct = tri(k.bwd_direct);
   }
   set_tuning(k);
 }

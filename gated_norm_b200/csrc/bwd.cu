@@ -1,4 +1,5 @@
 // bwd.cu -- instantiations and launcher of the backward kernel and of the dw second pass.
+#include "bwd_direct.cuh"
 #include "bwd_kernel.cuh"
 #include "launch.h"
 
@@ -21,7 +22,27 @@ static cudaError_t launch_bwd_geometry(const gnorm_plan& p, const BwdArgs& a,
                   : launch_bwd_weight<TPR, CPT, false>(p, a, stream, pdl);
 }
 
+template <int TPR>
+static cudaError_t launch_bwd_direct(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream,
+                                     bool pdl) {
+  if (a.w_fp32)
+    return launch_kernel(gated_rmsnorm_bwd_direct_kernel<TPR, true>, p.grid, kDirectThreads, 0,
+                         stream, pdl, a);
+  return launch_kernel(gated_rmsnorm_bwd_direct_kernel<TPR, false>, p.grid, kDirectThreads, 0,
+                       stream, pdl, a);
+}
+
 cudaError_t launch_bwd(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream, bool pdl) {
+  if (p.direct_loads) {
+    if (p.chunks_per_thread != 1) return cudaErrorInvalidConfiguration;
+    switch (p.threads_per_row) {
+      case 4: return launch_bwd_direct<4>(p, a, stream, pdl);
+      case 8: return launch_bwd_direct<8>(p, a, stream, pdl);
+      case 16: return launch_bwd_direct<16>(p, a, stream, pdl);
+      case 32: return launch_bwd_direct<32>(p, a, stream, pdl);
+      default: return cudaErrorInvalidConfiguration;
+    }
+  }
   const int key = p.threads_per_row * 8 + p.chunks_per_thread;
   switch (key) {
     case 4 * 8 + 1: return launch_bwd_geometry<4, 1>(p, a, stream, pdl);

@@ -41,6 +41,10 @@ GNORM_HD constexpr int max_ctas_per_sm(int kind, int threads_per_row, int chunks
 constexpr int kDirectThreads = 256;
 constexpr int kDirectRows = 2;
 constexpr int kDirectCtasPerSm = 4;
+// The backward's counterpart (gated_rmsnorm_bwd_direct_kernel) for very few rows per SM:
+// two rows per row group per iteration, 2 CTAs per SM (up to 128 registers per thread).
+constexpr int kDirectBwdRows = 2;
+constexpr int kDirectBwdCtasPerSm = 2;
 
 // Bytes one tensor of a pipeline stage occupies: R rows of N BF16 values, rounded up to
 // 128 bytes so every tensor of a stage starts 128-byte aligned (as tiled TMA copies require).

@@ -13,7 +13,8 @@
 // and within a tier: if the rows per CTA fit in one stage, one block per CTA; otherwise k
 // equal blocks per CTA, block size chosen so all CTAs get the same number of rows.  In the
 // forward's latency tier, rows of N <= 256 skip the staging altogether: 4 CTAs of 256
-// threads per SM load them straight into registers (gated_rmsnorm_fwd_direct_kernel).
+// threads per SM load them straight into registers (gated_rmsnorm_fwd_direct_kernel); so
+// does the backward of such rows under 256 KB of dy, x and g per SM (2 CTAs per SM).
 #include <algorithm>
 #include <cstdint>
 #include <cstring>
@@ -103,6 +104,33 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
     out->grid = static_cast<int>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * ctas));
     out->num_blocks = blocks;
     out->smem_bytes = 0;
+    out->direct_loads = 1;
+    return GNORM_OK;
+  }
+
+  // Backward of narrow rows with very few rows per SM: straight into registers as well.
+  const bool bwd_capable = kind == 1 && geo.chunks_per_thread == 1 && geo.threads_per_row <= 32;
+  const bool bwd_tier = rows_per_sm * (3 * N * 2) < kBwdDirectTierBytes;
+  if (bwd_capable && (g_knobs.bwd_direct == 1 || (g_knobs.bwd_direct == 0 && bwd_tier))) {
+    const int64_t rows_per_iter =
+        static_cast<int64_t>(kDirectThreads / geo.threads_per_row) * kDirectBwdRows;
+    const int ctas = std::min(kDirectBwdCtasPerSm, g_knobs.ctas_per_sm > 0
+                                                       ? g_knobs.ctas_per_sm
+                                                       : kDirectBwdCtasPerSm);
+    const int64_t blocks = ceil_div(M, rows_per_iter);
+    out->kind = 1;
+    out->threads_per_row = geo.threads_per_row;
+    out->chunks_per_thread = 1;
+    out->consumer_threads = kDirectThreads;
+    out->rows_per_stage = static_cast<int>(rows_per_iter);
+    out->stages = 0;
+    out->ctas_per_sm = ctas;
+    out->grid = static_cast<int>(std::min<int64_t>(blocks, static_cast<int64_t>(num_sms) * ctas));
+    out->num_blocks = blocks;
+    out->smem_bytes = 0;
+    out->dynamic_schedule = 0;  // rows are assigned statically in both modes
+    out->fused_reduce = 0;
+    out->partials = out->grid;
     out->direct_loads = 1;
     return GNORM_OK;
   }

@@ -23,6 +23,10 @@ constexpr int64_t kFwdLatencyStageBytes = 16384;
 constexpr int64_t kFwdLatencyTierBytes = 512 * 1024;
 constexpr int64_t kBwdStageBytes = 49152;
 constexpr int kBwdMinStageRows = 3;
+// Backward of rows of N <= 256 loaded straight into registers under this many bytes of dy,
+// x and g per SM (measured on B200: faster or equal up to ~220 rows per SM at N = 128, equal
+// at ~440, slower beyond).
+constexpr int64_t kBwdDirectTierBytes = 256 * 1024;
 // At most 3 backward stages in flight per SM: measured best or equal on every workload
 // (368640x128 backward 89.2 -> 83.1 us with 3 instead of 4 stages of ~48 KB).
 constexpr int kBwdMaxStages = 3;

@@ -276,7 +276,7 @@ typedef struct gnorm_plan {
   int fused_reduce;      /* 1: the last CTA to finish reduces the dw partials */
   int partials;          /* rows of the FP32 dw partial buffer (backward), else 0 */
   int l2_prefetch;       /* 1: warm L2 with the block each CTA loads after its ring's */
-  int direct_loads;      /* forward: 1 = rows loaded straight into registers, no staging
+  int direct_loads;      /* 1 = rows loaded straight into registers, no staging
                             (rows_per_stage = rows per CTA and iteration, stages = 0) */
 } gnorm_plan;
 
@@ -314,6 +314,8 @@ typedef struct gnorm_tuning {
   int chain_prefetch;    /* 1: in gnorm_ckpt_step, copy inputs before the previous kernel ends, 2: do not */
   int host_chunk_bytes;  /* gnorm_ckpt_step_host: bytes of x, g and dy per chunk */
   int fwd_direct;        /* forward of rows of N <= 256: 1 load straight into registers at any
+                            size, 2 always stage rows in shared memory (0: by rows per SM) */
+  int bwd_direct;        /* backward of rows of N <= 256: 1 load straight into registers at any
                             size, 2 always stage rows in shared memory (0: by rows per SM) */
 } gnorm_tuning;
 

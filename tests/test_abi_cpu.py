@@ -87,15 +87,23 @@ def test_plan_invariants(sms, kind):
                 p = gn.gnorm_plan_query(kind, M, N, det, sms)
                 R, G = p["rows_per_stage"], p["grid"]
                 rows_per_sm = -(-M // sms)
-                latency = rows_per_sm * 4 * N < 512 * 1024
-                assert p["direct_loads"] == (kind == 0 and N <= 256 and latency)
+                if kind == 0:
+                    direct = N <= 256 and rows_per_sm * 4 * N < 512 * 1024
+                else:
+                    direct = N <= 256 and rows_per_sm * 6 * N < 256 * 1024
+                assert p["direct_loads"] == direct
                 if p["direct_loads"]:  # rows straight into registers, no stages
                     tpr = p["threads_per_row"]
+                    ctas = 4 if kind == 0 else 2
                     assert p["chunks_per_thread"] == 1 and tpr * 8 >= N and tpr <= 32
                     assert p["consumer_threads"] == 256 and R == (256 // tpr) * 2
                     assert p["stages"] == 0 and p["smem_bytes"] == 0
                     assert p["num_blocks"] * R >= M and (p["num_blocks"] - 1) * R < M
-                    assert 1 <= G <= min(p["num_blocks"], 4 * sms) and p["ctas_per_sm"] == 4
+                    assert 1 <= G <= min(p["num_blocks"], ctas * sms)
+                    assert p["ctas_per_sm"] == ctas
+                    if kind == 1:  # static rows in both modes; one partial row per CTA
+                        assert p["partials"] == G and p["dynamic_schedule"] == 0
+                        assert p["fused_reduce"] == 0
                     continue
                 assert 1 <= R and p["stages"] >= 2
                 assert p["num_blocks"] * R >= M and (p["num_blocks"] - 1) * R < M
@@ -157,7 +165,7 @@ def test_tier_edge_rows_per_sm():
         assert wide_lat["ctas_per_sm"] == wide_stream["ctas_per_sm"] == 2
         assert wide_lat["rows_per_stage"] == 1 and wide_stream["rows_per_stage"] == 3
         try:
-            gn.gnorm_set_tuning(fwd_direct=2)  # the staged forward's blocks
+            gn.gnorm_set_tuning(fwd_direct=2, bwd_direct=2)  # the staged kernels' blocks
             for kind in (0, 1):
                 big = gn.gnorm_plan_query(kind, 1 << 12, N, True, sms)
                 ctas = sms * big["ctas_per_sm"]
@@ -194,8 +202,8 @@ def test_ctas_per_sm_never_exceeds_the_compiled_residency():
                     fit = 1 if p["consumer_threads"] > 256 else (
                         (3 if cpt == 1 else 2 if cpt <= 4 else 1) if kind == 0 else
                         (2 if cpt == 1 else 1))
-                    if p["direct_loads"]:
-                        fit = 4  # the direct-load forward's compiled residency
+                    if p["direct_loads"]:  # the direct-load kernels' compiled residency
+                        fit = 4 if kind == 0 else 2
                     assert p["ctas_per_sm"] <= fit
 
 

@@ -28,6 +28,8 @@ KNOB_SETS = [
     dict(ctas_per_sm=2, stage_bytes=98304),
     dict(fwd_direct=1),
     dict(fwd_direct=2),
+    dict(bwd_direct=1),
+    dict(bwd_direct=2),
 ]
 
 
@@ -62,11 +64,11 @@ def test_knobs_do_not_change_results(M, N, det):
                                  (70001, 128)])
 @pytest.mark.parametrize("w_fp32", [False, True])
 @pytest.mark.parametrize("strided", [False, True])
-def test_direct_and_staged_forward_agree(M, N, w_fp32, strided):
-    """The forward that loads rows straight into registers and the one that stages them in
-    shared memory do the same arithmetic in the same order: bitwise equal y and rstd, for
-    packed and strided rows (x and g as the column halves of one buffer) and both weight
-    types."""
+def test_direct_and_staged_kernels_agree(M, N, w_fp32, strided):
+    """The kernels that load rows straight into registers and the ones that stage them in
+    shared memory do the same arithmetic in the same order: bitwise equal y, rstd, dx and dg,
+    for packed and strided rows (x and g as the column halves of one buffer) and both weight
+    types; dw (summed in another order) within its tolerance."""
     case = Case(M, N, seed=29)
     if strided:
         xg = torch.cat([case.x, case.g], dim=1)
@@ -84,4 +86,24 @@ def test_direct_and_staged_forward_agree(M, N, w_fp32, strided):
     finally:
         gn.gnorm_set_tuning()
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    # the backward likewise: dx and dg bitwise equal, dw within its tolerance of the oracle
+    dy = case.dy
+    if strided:
+        dyz = torch.cat([case.dy, torch.zeros_like(case.dy)], dim=1)
+        dy = dyz[:, :N]
+    rstd = outs[0][1]
+    bwd = []
+    try:
+        for mode in (1, 2):
+            gn.gnorm_set_tuning(bwd_direct=mode)
+            assert gn.gnorm_plan_query(1, M, N, True, 148)["direct_loads"] == (mode == 1)
+            bwd.append(gn.gnorm_bwd(dy, x, g, w, rstd, dw_fp32=True, deterministic=True))
+        torch.cuda.synchronize()
+    finally:
+        gn.gnorm_set_tuning()
+    assert torch.equal(bwd[0][0], bwd[1][0]) and torch.equal(bwd[0][1], bwd[1][1])
+    dw_ref = case.oracle_dw()
+    for out in bwd:
+        rep = dw_fp32_check(dev_to_f64(out[2]), dw_ref)
+        assert rep["ok"], rep
     assert gn.gnorm_device_error(reset=True) == 0
