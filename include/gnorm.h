@@ -19,17 +19,21 @@
  *   - Tensors are row-major and contiguous ("packed" rows): element (m, j) of an [M, N]
  *     tensor sits at index m*N + j.  x, g, w, y, dy, dx, dg are BF16 (IEEE bfloat16 bit
  *     patterns, 2 bytes); rstd is FP32; dw is BF16 or FP32 (dw_fp32).
- *   - All tensor pointers are DEVICE pointers of the current CUDA device.  Every pointer
- *     except rstd must be 16-byte aligned; rstd must be 4-byte aligned.
+ *   - All tensor pointers are DEVICE pointers of the current CUDA device (except for
+ *     gnorm_ckpt_step_host, which takes host buffers).  Every pointer except rstd must be
+ *     16-byte aligned; rstd must be 4-byte aligned.
  *   - N must be a multiple of 8 with 8 <= N <= GNORM_N_MAX.  M >= 0; M == 0 is a no-op
  *     for the forward, and the backward then writes dw = 0.  When M == 0 the per-row
  *     tensors may be NULL.
  *   - eps must be finite and >= 0.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls only enqueue
  *     work: they never synchronise, never allocate and are safe to capture in a CUDA
- *     graph.  Each call is launched with programmatic dependent launch, so a kernel of
- *     this library may start its prologue while the previous kernel on the stream drains;
- *     it reads and writes global memory only after that kernel has completed.
+ *     graph (gnorm_ckpt_step_host excepted; see there).  Each kernel is launched with
+ *     programmatic dependent launch, so it may start its prologue while the previous
+ *     kernel on the stream drains; it reads and writes global memory only after that
+ *     kernel has completed -- except that inside gnorm_ckpt_step the second forward and
+ *     the backward may start reading x, g and dy early, which their predecessors in the
+ *     same call never write.
  *   - The caller owns every buffer; the library keeps no pointer after a call returns.
  *   - Outputs must not overlap any input or each other (GNORM_ERR_ALIAS).
  *   - Errors are detected on the host before any launch and returned as a gnorm_status;
