@@ -36,8 +36,10 @@ def _strided_layout(case):
                 dx=grad[:, :N], dg=grad[:, N:2 * N], grad=grad)
 
 
-# (4099, 136), (33, 256), (257, 128): strided blocks load through 2-D tensor maps;
-# (65, 4096) and (300000, 8) (more than 256 rows per block) through one copy per row.
+# With the default plans, narrow rows with few rows per SM take the direct-load kernels
+# (strided rows are plain loads there); (50000, 128)'s backward stages its blocks through
+# 2-D tensor maps and (65, 4096) through one copy per row.  The staged kernels' strided
+# paths at the other sizes are compared with the direct ones in test_knobs_gpu.py.
 @pytest.mark.parametrize("M,N", [(1, 128), (257, 128), (4099, 136), (33, 256), (65, 4096),
                                  (300000, 8), (50000, 128)])
 @pytest.mark.parametrize("det", [True, False])
