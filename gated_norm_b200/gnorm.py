@@ -84,7 +84,7 @@ def gnorm_selftest_wait_timeout(timeout_us: int = 20000) -> int:
 def gnorm_set_tuning(**knobs) -> None:
     """Process-wide experiment knobs (fields of gnorm_tuning; 0 = built-in).  No arguments
     restores every built-in choice.  Tri-state knobs (l2_prefetch, tail_reduce,
-    chain_prefetch): 1 on, 2 off, 0 built-in."""
+    chain_prefetch, fwd_direct, bwd_direct): 1 on, 2 off, 0 built-in."""
     t = GnormTuning()
     names = {f for f, _ in GnormTuning._fields_}
     for k, v in knobs.items():
