@@ -146,6 +146,13 @@ def _weight(w, N, device):
     return 1 if w.dtype == torch.float32 else 0
 
 
+def _device_buffer(t, name: str, device):
+    """Scratch handed to the library: contiguous memory on the device that runs the call
+    (a host buffer here would reach a kernel as a device pointer)."""
+    if t.device != torch.device(device) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous tensor on {device}")
+
+
 def _check(st: int, where: str):
     if st != GNORM_OK:
         raise GnormError(st, where)
@@ -235,6 +242,8 @@ def _bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic, ws):
         _vec(dw, N, (dw_dtype,), "dw", x.device)
     if ws is None:
         ws = workspace(M, N, deterministic, x.device)
+    else:
+        _device_buffer(ws, "workspace_buf", x.device)
     d = GnormBwdDesc(dy=_ptr(dy), lddy=lddy, x=_ptr(x), ldx=ldx, g=_ptr(g), ldg=ldg, w=_ptr(w),
                      w_fp32=w_fp32, rstd=_ptr(rstd), dx=_ptr(dx), lddx=lddx, dg=_ptr(dg),
                      lddg=lddg, dw=_ptr(dw), dw_fp32=int(bool(dw_fp32)),
@@ -308,8 +317,9 @@ def gnorm_ckpt_step_host(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None,
     if w.device.type != "cpu" or w.dtype != torch.bfloat16 or tuple(w.shape) != (N,):
         raise ValueError(f"w must be a BF16 [{N}] CPU tensor")
     pin = x.is_pinned()
-    device = torch.device("cuda", torch.cuda.current_device()) if device is None \
-        else torch.device(device)
+    device = torch.device("cuda") if device is None else torch.device(device)
+    if device.index is None:
+        device = torch.device("cuda", torch.cuda.current_device())
 
     def new(shape, dtype):
         return torch.empty(shape, dtype=dtype, pin_memory=pin)
@@ -328,6 +338,8 @@ def gnorm_ckpt_step_host(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None,
     with torch.cuda.device(device):
         if dev_buf is None:
             dev_buf = _host_step_buffer(M, N, deterministic, device)
+        else:
+            _device_buffer(dev_buf, "dev_buf", device)
         st = lib.gnorm_ckpt_step_host(_ptr(x), _ptr(g), _ptr(w), float(eps), _ptr(dy), _ptr(y),
                                       _ptr(rstd), _ptr(dx), _ptr(dg), _ptr(dw),
                                       int(bool(dw_fp32)), int(bool(deterministic)), M, N,
@@ -339,7 +351,8 @@ def gnorm_ckpt_step_host(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None,
 
 def gnorm_dw_reduce(partials, *, dw=None, dw_fp32: bool = True, stream=None):
     """Fixed-order sum of FP32 partial rows [P, N] into dw [N] (BF16 or FP32)."""
-    if partials.dtype != torch.float32 or partials.dim() != 2 or not partials.is_contiguous():
+    if (partials.device.type != "cuda" or partials.dtype != torch.float32 or
+            partials.dim() != 2 or not partials.is_contiguous()):
         raise ValueError("partials must be a contiguous FP32 [P, N] CUDA tensor")
     P, N = partials.shape
     dw_dtype = torch.float32 if dw_fp32 else torch.bfloat16
