@@ -1,25 +1,27 @@
 """Benchmark of the SiLU-gated RMSNorm training step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload NAME] [--nondeterministic] [--dw-fp32]
+                    [--workload NAME] [--nondeterministic] [--dw-bf16] [--flush]
 
 A step is one checkpointed training step over one batch of seeded synthetic rows:
 forward, forward again (recompute), backward with the dw reduction -- every stage of the
-path -- replayed from one CUDA graph ("ckptg").  Each timed step also replays the backward
-("bwdg") and the forward ("fwdg") alone, each from its own graph, for the per-operation
-times and the roofline of the dominant kernel (the forward: two launches per step, the
-largest share of the step's device time).  The default workload is 65536 x 128 (a
-per-head gated norm of a linear-attention output, 512 heads x 128 tokens).  Times are
-CUDA-event device times on the launching stream; L2 is flushed (256 MiB write) before
-every timed replay, outside the events.  `value` is the checkpointed step's algorithmic
-HBM bytes of the whole job / the max-over-ranks summed step time (GB/s).
+path -- replayed from one CUDA graph ("ckptg").  The default workload is 262144 x 256 with
+an FP32 dw, deterministic (the checkpointed step with FP32 dw, "stepg_f32" in the pages'
+list of operations).  The timed region is K steps.  When the inputs are larger than L2
+(x and g alone exceed it at every large workload) the K replays run back to back between
+one pair of CUDA events; otherwise L2 is flushed before every replay, outside a pair of
+events around that replay.  After the timed region the forward ("fwdg") and the backward
+("bwdg") are timed the same way from their own graphs, for the per-operation times and the
+roofline of each; the three operations are also timed with a cold L2 before every replay
+(`us_per_call_cold_l2`), and `per_config` gives fwdg / bwdg / ckptg of the other large
+workloads.  `value` is the checkpointed step's algorithmic HBM bytes of the whole job / the
+max-over-ranks time of the K steps (GB/s).
 
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the
 data path; the rows of a data-parallel batch are independent).  `--impl reference` times
 the FP64 CPU oracle on a bounded sample of the same workload (rank 0 only).  `--floor`
-adds, after the timed region, the same measurement of an empty graph and of torch
-elementwise kernels that move the forward's and backward's main streams (context for the
-fixed per-launch cost at small sizes).
+adds the same measurement of an empty graph and of torch elementwise kernels that move the
+forward's and backward's main streams.
 """
 from __future__ import annotations
 
@@ -42,7 +44,8 @@ sys.path.insert(0, ROOT)
 from synthetic import WORKLOADS, bf16_bits_to_f64, make_inputs  # noqa: E402
 
 METRIC = "fwd / bwd / ckpt-step µs and achieved HBM GB/s (% of B200 roofline), 1 GPU"
-DEFAULT_WORKLOAD = "linattn_65536x128"
+DEFAULT_WORKLOAD = "mid_262144x256"
+PER_CONFIG_WORKLOADS = ("long_368640x128", "wide_16384x4096", "mid_262144x256")
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
 
@@ -272,7 +275,7 @@ def run_reference(args, wl):
     for _ in range(args.steps):
         oracle.ckpt_step(x, g, w, wl.eps, dy)
     el = time.perf_counter() - t0
-    value = ckpt_bytes(rows, wl.N, args.dw_fp32) * args.steps / el / 1e9
+    value = ckpt_bytes(rows, wl.N, not args.dw_bf16) * args.steps / el / 1e9
     sample = f"{rows} of {wl.M} rows x N={wl.N} per step (FP64 numpy oracle, one core)"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
@@ -291,45 +294,160 @@ def run_reference(args, wl):
 
 # ----------------------------------------------------------------------------- our leg
 
-def measure_floor(torch, dev, stream, flush, x, g, dy, y, dx, K):
+def l2_bytes(torch, dev):
+    try:
+        return int(torch.cuda.get_device_properties(dev).L2_cache_size)
+    except Exception:
+        return 126 * 1000 * 1000
+
+
+def capture_graph(torch, dev, stream, fn, launches=1):
+    """A CUDA graph holding `launches` consecutive calls of `fn` (captured on a side stream
+    after two eager calls, which also set up any per-device state)."""
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        fn()
+        fn()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        for _ in range(launches):
+            fn()
+    return graph
+
+
+class Timer:
+    """CUDA-event timing of graph replays on `stream`.
+
+    streamed=True: the replays run back to back between one pair of events (the inputs of
+    every operation are larger than L2, so one replay finds nothing of the previous one's
+    rows in L2); the per-replay time is the total over the count.
+    streamed=False: L2 is flushed (a write of `flush`, larger than L2) before every replay,
+    outside a pair of events around that replay."""
+
+    def __init__(self, torch, stream, flush, streamed):
+        self.torch, self.stream, self.flush, self.streamed = torch, stream, flush, streamed
+
+    def run(self, graph, reps):
+        """Total device milliseconds of `reps` replays, and the per-replay list (for the
+        streamed mode, each replay's own events sit inside the outer pair)."""
+        torch, s = self.torch, self.stream
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        if self.streamed:
+            a0, b0 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a0.record(s)
+            for _ in range(reps):
+                graph.replay()
+            b0.record(s)
+            torch.cuda.synchronize()
+            return a0.elapsed_time(b0), None
+        for a, b in ev:
+            self.flush.zero_()
+            a.record(s)
+            graph.replay()
+            b.record(s)
+        torch.cuda.synchronize()
+        per = [a.elapsed_time(b) for a, b in ev]
+        return float(sum(per)), per
+
+    def cold(self, graph, reps):
+        """Mean ms of `reps` replays each after an L2 flush (events around each replay)."""
+        saved = self.streamed
+        self.streamed = False
+        try:
+            total, _ = self.run(graph, reps)
+        finally:
+            self.streamed = saved
+        return total / reps
+
+
+def measure_floor(torch, dev, stream, timer, x, g, dy, y, dx, reps):
     """The timing method's own floor: an empty graph (one one-element add) and torch
     elementwise kernels over the same [M, N] BF16 tensors -- y = x * g (the forward's
-    reads and write) and dx = x + g * dy (three reads, one write) -- each replayed from a
-    CUDA graph between the same L2 flush and events as the timed steps."""
+    reads and write) and dx = x + g * dy (three reads, one write) -- timed exactly as the
+    operations are."""
     one = torch.zeros(1, device=dev)
     ops = {
         "empty_graph": (0, lambda: one.add_(1)),
         "torch_mul": (3 * x.numel() * 2, lambda: torch.mul(x, g, out=y)),
         "torch_addcmul": (4 * x.numel() * 2, lambda: torch.addcmul(x, g, dy, out=dx)),
     }
-    reps = max(20, min(K, 200))
     out = {}
     for name, (nbytes, fn) in ops.items():
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            fn()
-            fn()
-        stream.wait_stream(side)
-        torch.cuda.synchronize(dev)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=side):
-            fn()
-        for _ in range(3):
-            flush.zero_()
-            graph.replay()
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-               for _ in range(reps)]
-        for a, b in evs:
-            flush.zero_()
-            a.record(stream)
-            graph.replay()
-            b.record(stream)
-        torch.cuda.synchronize(dev)
-        t_us = statistics.mean(a.elapsed_time(b) * 1e3 for a, b in evs)
+        graph = capture_graph(torch, dev, stream, fn)
+        timer.run(graph, 3)
+        total, _ = timer.run(graph, reps)
+        t_us = total / reps * 1e3
         out[name] = {"us": t_us, "bytes": nbytes,
                      "gbs": (nbytes / (t_us * 1e-6) / 1e9) if nbytes else None}
         del graph
+    return out
+
+
+class Problem:
+    """Device tensors of one workload and CUDA graphs of its three operations (fwdg, bwdg,
+    ckptg, as the pages name them)."""
+
+    def __init__(self, torch, gn, dev, stream, wl, det, fp32, seed_offset=0, graphs=True):
+        self.torch, self.gn, self.wl = torch, gn, wl
+        self.M, self.N, self.eps = wl.M, wl.N, wl.eps
+        self.det, self.fp32 = det, fp32
+        d = make_inputs(wl.M, wl.N, seed=wl.seed + seed_offset, g_std=wl.g_std,
+                        outlier_frac=wl.outlier_frac, outlier_scale=wl.outlier_scale)
+
+        def dev_bf16(bits):
+            return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+
+        self.x, self.g, self.dy, self.w = (dev_bf16(d[k]) for k in ("x", "g", "dy", "w"))
+        self.y, self.dx, self.dg = (torch.empty_like(self.x) for _ in range(3))
+        self.rstd = torch.empty(wl.M, dtype=torch.float32, device=dev)
+        self.dw = torch.empty(wl.N, dtype=torch.float32 if fp32 else torch.bfloat16, device=dev)
+        self.ws = torch.zeros(max(gn.gnorm_bwd_workspace_bytes(wl.M, wl.N, det), 256),
+                              dtype=torch.uint8, device=dev)
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.plan_f = gn.gnorm_plan_query(0, wl.M, wl.N, det, sms)
+        self.plan_b = gn.gnorm_plan_query(1, wl.M, wl.N, det, sms)
+        self.bwd_launches = 1 + (0 if self.plan_b["fused_reduce"] else 1)
+        self.launches = {"ckpt": 2 + self.bwd_launches, "bwd": self.bwd_launches, "fwd": 1}
+        self.graphs = {name: capture_graph(torch, dev, stream, fn)
+                       for name, fn in (("ckpt", self.op_ckpt), ("bwd", self.op_bwd),
+                                        ("fwd", self.op_fwd))} if graphs else {}
+
+    def op_fwd(self):
+        self.gn.gnorm_fwd(self.x, self.g, self.w, self.eps, y=self.y, rstd=self.rstd)
+
+    def op_bwd(self):
+        self.gn.gnorm_bwd(self.dy, self.x, self.g, self.w, self.rstd, dx=self.dx, dg=self.dg,
+                          dw=self.dw, dw_fp32=self.fp32, deterministic=self.det,
+                          workspace_buf=self.ws)
+
+    def op_ckpt(self):
+        self.gn.gnorm_ckpt_step(self.x, self.g, self.w, self.eps, self.dy, y=self.y,
+                                rstd=self.rstd, dx=self.dx, dg=self.dg, dw=self.dw,
+                                dw_fp32=self.fp32, deterministic=self.det, workspace_buf=self.ws)
+
+    def fwd_kernel(self):
+        return ("gated_rmsnorm_fwd_direct_kernel" if self.plan_f["direct_loads"]
+                else "gated_rmsnorm_fwd_kernel")
+
+    def bytes(self):
+        return {"fwd": fwd_bytes(self.M, self.N), "bwd": bwd_bytes(self.M, self.N, self.fp32),
+                "ckpt": ckpt_bytes(self.M, self.N, self.fp32)}
+
+    def release(self):
+        self.graphs.clear()
+
+
+def op_times(timer, prob, reps):
+    """Mean device microseconds per replay of fwdg, bwdg and ckptg."""
+    out = {}
+    for name in ("fwd", "bwd", "ckpt"):
+        timer.run(prob.graphs[name], 3)
+        total, _ = timer.run(prob.graphs[name], reps)
+        out[name] = total / reps * 1e3
     return out
 
 
@@ -345,111 +463,89 @@ def run_ours(args, wl):
         dist = init_dist(dev, "nccl")
     import gated_norm_b200 as gn
 
-    M, N, eps = wl.M, wl.N, wl.eps
+    knobs = parse_tune(args.tune)
+    if knobs:
+        gn.gnorm_set_tuning(**knobs)
     det = not args.nondeterministic
-    fp32 = args.dw_fp32
-    d = make_inputs(M, N, seed=wl.seed + rank, g_std=wl.g_std, outlier_frac=wl.outlier_frac)
-
-    def dev_bf16(bits):
-        return torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
-
-    x, g, dy, w = (dev_bf16(d[k]) for k in ("x", "g", "dy", "w"))
-    y, dx, dg = (torch.empty_like(x) for _ in range(3))
-    rstd = torch.empty(M, dtype=torch.float32, device=dev)
-    dw = torch.empty(N, dtype=torch.float32 if fp32 else torch.bfloat16, device=dev)
-    ws = torch.zeros(max(gn.gnorm_bwd_workspace_bytes(M, N, det), 256), dtype=torch.uint8,
-                     device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    fp32 = not args.dw_bf16
     stream = torch.cuda.current_stream(dev)
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    plan_f = gn.gnorm_plan_query(0, M, N, det, sms)
-    plan_b = gn.gnorm_plan_query(1, M, N, det, sms)
-    fwd_kernel = ("gated_rmsnorm_fwd_direct_kernel" if plan_f["direct_loads"]
-                  else "gated_rmsnorm_fwd_kernel")
-    bwd_launches = 1 + (0 if plan_b["fused_reduce"] else 1)
-
-    # The operations as the pages time them: each replayed from its own CUDA graph.
-    def op_fwd():
-        gn.gnorm_fwd(x, g, w, eps, y=y, rstd=rstd)
-
-    def op_bwd():
-        gn.gnorm_bwd(dy, x, g, w, rstd, dx=dx, dg=dg, dw=dw, dw_fp32=fp32, deterministic=det,
-                     workspace_buf=ws)
-
-    def op_ckpt():
-        gn.gnorm_ckpt_step(x, g, w, eps, dy, y=y, rstd=rstd, dx=dx, dg=dg, dw=dw, dw_fp32=fp32,
-                           deterministic=det, workspace_buf=ws)
-
-    def capture(fn):
-        side = torch.cuda.Stream(dev)
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            fn()
-            fn()
-        stream.wait_stream(side)
-        torch.cuda.synchronize(dev)
-        graph = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(graph, stream=side):
-            fn()
-        return graph
-
-    graphs = {"ckpt": capture(op_ckpt), "bwd": capture(op_bwd), "fwd": capture(op_fwd)}
-    launches = {"ckpt": 2 + bwd_launches, "bwd": bwd_launches, "fwd": 1}
-    order = ("ckpt", "bwd", "fwd")
-
-    def one_step(evs=None):
-        # one timed step: the checkpointed step (the measured unit), then the backward and
-        # the forward alone for the per-operation times; L2 is flushed before each, outside
-        # the events.
-        for j, name in enumerate(order):
-            flush.zero_()
-            if evs:
-                evs[2 * j].record(stream)
-            graphs[name].replay()
-            if evs:
-                evs[2 * j + 1].record(stream)
+    l2 = l2_bytes(torch, dev)
+    flush = torch.empty(max(L2_FLUSH_BYTES, 2 * l2), dtype=torch.uint8, device=dev)
+    prob = Problem(torch, gn, dev, stream, wl, det, fp32, seed_offset=rank)
+    M, N = prob.M, prob.N
+    # The smallest operation's inputs: the forward reads x and g.
+    streamed = (not args.flush) and 2 * M * N * 2 > l2
+    timer = Timer(torch, stream, flush, streamed)
+    ckpt_graph = prob.graphs["ckpt"]
 
     for _ in range(args.warmup):
-        one_step()
+        if not streamed:
+            flush.zero_()
+        ckpt_graph.replay()
     torch.cuda.synchronize()
 
     K = args.steps
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(K)]
     clocks = ClockSampler(local)
     if rank == 0:
         clocks.start()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(K):
-        one_step(evs[i])
+    total_ms, per_step = timer.run(ckpt_graph, K)   # the timed region: K checkpointed steps
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    clk = clocks.stop() if rank == 0 else None
-
-    t_ckpt = [evs[i][0].elapsed_time(evs[i][1]) for i in range(K)]
-    t_bwd = [evs[i][2].elapsed_time(evs[i][3]) for i in range(K)]
-    t_fwd = [evs[i][4].elapsed_time(evs[i][5]) for i in range(K)]
-    total_ms = max_over_ranks(float(sum(t_ckpt)), world, dev)
+    total_ms = max_over_ranks(total_ms, world, dev)
     step_bytes = ckpt_bytes(M, N, fp32)
     value = whole_job_gbs(step_bytes, K, world, total_ms)
     peak, peak_kind = measured_peaks()
 
-    # one checkpointed step through the single public entry point, host buffers in and out
+    # the forward and the backward alone, timed the same way (their own graphs)
+    us = op_times(timer, prob, K)
+    us["ckpt"] = total_ms / K * 1e3
+    # the same operations with a cold L2 before every replay, events around each replay
+    # (this also counts each replay's own launch latency)
+    cold_reps = max(10, min(K, 100))
+    us_cold = {name: prob_t * 1e3 for name, prob_t in
+               ((n, timer.cold(prob.graphs[n], cold_reps)) for n in ("fwd", "bwd", "ckpt"))}
+    per_config = {}
+    if args.per_config and world == 1:
+        for name in PER_CONFIG_WORKLOADS:
+            if name == wl.name:
+                continue
+            other = Problem(torch, gn, dev, stream, WORKLOADS[name], det, fp32)
+            o_streamed = (not args.flush) and 2 * other.M * other.N * 2 > l2
+            o_timer = Timer(torch, stream, flush, o_streamed)
+            t = op_times(o_timer, other, args.per_config_steps)
+            b = other.bytes()
+            per_config[name] = {
+                "M": other.M, "N": other.N, "us": t,
+                "gbs": {k: b[k] / (t[k] * 1e-6) / 1e9 for k in t},
+                "frac_of_peak": {k: b[k] / (t[k] * 1e-6) / 1e9 / peak for k in t},
+                "fwd_kernel": other.fwd_kernel(),
+                "l2": "inputs larger than L2, replays back to back" if o_streamed
+                      else "L2 flushed before every replay",
+            }
+            other.release()
+            del other
+            torch.cuda.synchronize()
+    clk = clocks.stop() if rank == 0 else None
+
+    # one checkpointed step through the public host-buffer entry point: inputs copied in
+    # and outputs copied back every step
     e2e = None
     if args.e2e_steps > 0:
-        hx, hg, hdy, hw = (t.cpu().pin_memory() for t in (x, g, dy, w))
+        hx, hg, hdy, hw = (t.cpu().pin_memory() for t in (prob.x, prob.g, prob.dy, prob.w))
         hy, hr, hdx, hdg, hdw = (torch.empty_like(t, device="cpu").pin_memory()
-                                 for t in (y, rstd, dx, dg, dw))
+                                 for t in (prob.y, prob.rstd, prob.dx, prob.dg, prob.dw))
         h2d = sum(t.numel() * t.element_size() for t in (hx, hg, hdy, hw))
         d2h = sum(t.numel() * t.element_size() for t in (hy, hr, hdx, hdg, hdw))
         dev_buf = torch.empty(gn.gnorm_ckpt_step_host_bytes(M, N, det), dtype=torch.uint8,
                               device=dev)
 
         def e2e_step():
-            gn.gnorm_ckpt_step_host(hx, hg, hw, eps, hdy, y=hy, rstd=hr, dx=hdx, dg=hdg, dw=hdw,
-                                    dw_fp32=fp32, deterministic=det, dev_buf=dev_buf,
+            gn.gnorm_ckpt_step_host(hx, hg, hw, prob.eps, hdy, y=hy, rstd=hr, dx=hdx, dg=hdg,
+                                    dw=hdw, dw_fp32=fp32, deterministic=det, dev_buf=dev_buf,
                                     device=dev, stream=stream)
 
         for _ in range(3):
@@ -468,46 +564,25 @@ def run_ours(args, wl):
                "path": "gnorm_ckpt_step_host: pinned host inputs and outputs; the library "
                        "copies each step's inputs in and outputs back, chunk by chunk, "
                        "overlapping both directions of the host link with the kernels"}
+        del dev_buf
 
-    # the forward launched eagerly (no graph), same flush and events, after the timed region
-    fwd_eager = []
-    for i in range(min(K, 200) + 3):
-        flush.zero_()
-        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_ev.record(stream)
-        op_fwd()
-        b_ev.record(stream)
-        fwd_eager.append((a_ev, b_ev))
-    torch.cuda.synchronize(dev)
-    fwd_eager_us = statistics.mean(a_ev.elapsed_time(b_ev) for a_ev, b_ev in fwd_eager[3:]) * 1e3
-
-    floor = measure_floor(torch, dev, stream, flush, x, g, dy, y, dx, K) if args.floor else None
+    floor = (measure_floor(torch, dev, stream, timer, prob.x, prob.g, prob.dy, prob.y, prob.dx,
+                           max(20, min(K, 200))) if args.floor else None)
 
     if world > 1:
         dist.barrier()
+        prob.release()
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
-    def avg(v):
-        return float(sum(v) / len(v))
-
-    us = {"fwd": avg(t_fwd) * 1e3, "bwd": avg(t_bwd) * 1e3, "ckpt": avg(t_ckpt) * 1e3}
-
-    def median_of_rounds(v, rounds=10):
-        n = max(1, len(v) // rounds)
-        meds = [statistics.median(v[i:i + n]) for i in range(0, n * (len(v) // n), n)]
-        return statistics.median(meds) * 1e3
-
-    us_median = {"fwd": median_of_rounds(t_fwd), "bwd": median_of_rounds(t_bwd),
-                 "ckpt": median_of_rounds(t_ckpt)}
-    gbs = {"fwd": fwd_bytes(M, N) / (us["fwd"] * 1e-6) / 1e9,
-           "bwd": bwd_bytes(M, N, fp32) / (us["bwd"] * 1e-6) / 1e9,
-           "ckpt": step_bytes / (us["ckpt"] * 1e-6) / 1e9}
+    b = prob.bytes()
+    gbs = {k: b[k] / (us[k] * 1e-6) / 1e9 for k in us}
+    gbs_cold = {k: b[k] / (us_cold[k] * 1e-6) / 1e9 for k in us_cold}
     fwd_traffic = profiled_traffic("fwd_kernel", wl.name)
     bwd_traffic = profiled_traffic("bwd_kernel", wl.name)
-    # device time of one step by kernel, from the standalone replays: the forward kernel
-    # (twice) and the backward operation (kernel + second pass)
+    # device time of one step by operation, from the standalone replays: the forward
+    # kernel (twice) and the backward operation (kernel + second pass)
     step_us = 2 * us["fwd"] + us["bwd"]
     shares = {"fwd_kernel_x2": 2 * us["fwd"] / step_us, "bwd_op": us["bwd"] / step_us}
     cpu = cpu_all = None
@@ -522,45 +597,98 @@ def run_ours(args, wl):
                        "sample": f"{a_procs} processes, each {a_rows} rows x N={N} of its own, "
                                  f"checkpointed steps for {args.cpu_seconds:.0f} s "
                                  "(FP64 numpy oracle, one process per core)"}
+    l2_note = (f"inputs larger than L2 ({2 * M * N * 2 / 1e6:.0f} MB of x and g per forward "
+               f"against {l2 / 1e6:.0f} MB of L2): replays back to back, no flush"
+               if streamed else
+               f"L2 flushed before every replay ({flush.numel() >> 20} MiB write, outside "
+               "the timed events)")
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "M": M, "N": N, "eps": eps,
-                   "step": "checkpointed step as one CUDA graph: fwd, fwd (recompute), bwd + dw reduction",
+        "config": {"workload": wl.name, "M": M, "N": N, "eps": prob.eps,
+                   "step": "checkpointed step as one CUDA graph: fwd, fwd (recompute), "
+                           "bwd + dw reduction",
                    "deterministic": det, "dw": "fp32" if fp32 else "bf16",
-                   "l2": "flushed between steps (256 MiB write, outside the timed events)",
-                   "parallelism": f"dp{world} (independent rows per rank, no collective)"},
+                   "l2": l2_note,
+                   "parallelism": f"dp{world} (independent rows per rank, no collective)",
+                   **({"tuning": knobs} if knobs else {})},
         "us_per_call": us,
-        "us_median_of_round_medians": us_median,
-        "us_fwd_eager": fwd_eager_us,
-        "timing": "fwd, bwd, ckpt each replayed from its own CUDA graph (fwdg, bwdg, ckptg)",
+        "timing": ("ckptg replayed K times back to back between two CUDA events (the timed "
+                   "region); fwdg and bwdg then timed the same way from their own graphs"
+                   if streamed else
+                   "each of ckptg, fwdg, bwdg replayed from its own CUDA graph between two "
+                   "CUDA events after an L2 flush"),
         "gbs": gbs,
         "frac_of_peak": {k: v / peak for k, v in gbs.items()},
+        "us_per_call_cold_l2": us_cold,
+        "frac_of_peak_cold_l2": {k: v / peak for k, v in gbs_cold.items()},
+        "cold_l2_note": (f"{cold_reps} replays each after a {flush.numel() >> 20} MiB L2 flush, "
+                         "events around each replay, so each also counts its graph's launch "
+                         "latency"),
         "roofline": {"bound": "hbm",
-                     "kernel": f"{fwd_kernel} (one launch per fwdg replay)",
+                     "kernel": f"{prob.fwd_kernel()} (one launch per fwdg replay)",
                      "achieved": gbs["fwd"], "peak": peak, "peak_kind": peak_kind,
                      "unit": "GB/s", "frac": gbs["fwd"] / peak,
-                     "algorithmic_bytes_per_launch": fwd_bytes(M, N),
+                     "algorithmic_bytes_per_launch": b["fwd"],
                      "traffic": fwd_traffic},
         "roofline_bwd": {"bound": "hbm",
                          "kernel": "gnorm_bwd (backward kernel + dw second pass, one bwdg "
                                    "replay)",
                          "achieved": gbs["bwd"], "peak": peak, "peak_kind": peak_kind,
                          "unit": "GB/s", "frac": gbs["bwd"] / peak,
-                         "algorithmic_bytes_per_launch": bwd_bytes(M, N, fp32),
+                         "algorithmic_bytes_per_launch": b["bwd"],
                          "traffic": bwd_traffic},
         "step_shares": shares,
+        "per_config": per_config or None,
         "cpu_baseline": cpu,
         "cpu_baseline_all_cores": cpu_all,
         "e2e": e2e,
-        "gpu_launches": sum(launches.values()) * K,
+        "gpu_launches": prob.launches["ckpt"] * K,
         "clocks": clk,
     }
     if floor is not None:
         line["floor"] = floor
     print(json.dumps(line))
     return 0
+
+
+def parse_tune(items):
+    """--tune KNOB=VALUE pairs -> a dict of gnorm_tuning fields."""
+    out = {}
+    for it in items:
+        k, _, v = it.partition("=")
+        if not k or not v:
+            raise SystemExit(f"bench.py: --tune wants KNOB=VALUE, got {it!r}")
+        out[k.strip()] = int(v)
+    return out
+
+
+def run_profile(args, wl):
+    """Only `--profile-op` on the workload's inputs: one untimed call, then `--reps` calls,
+    nothing else on the GPU (a short, fixed launch list for ncu captures)."""
+    import torch
+
+    import gated_norm_b200 as gn
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    knobs = parse_tune(args.tune)
+    if knobs:
+        gn.gnorm_set_tuning(**knobs)
+    prob = Problem(torch, gn, dev, torch.cuda.current_stream(dev), wl,
+                   not args.nondeterministic, not args.dw_bf16, graphs=False)
+    fn = {"fwd": prob.op_fwd, "bwd": prob.op_bwd, "ckpt": prob.op_ckpt}[args.profile_op]
+    torch.cuda.synchronize()
+    for _ in range(args.reps):
+        fn()
+    torch.cuda.synchronize()
+    err = gn.gnorm_device_error(reset=True)
+    prob.release()
+    print(json.dumps({"profile_op": args.profile_op, "workload": wl.name, "reps": args.reps,
+                      "tune": knobs, "plan_fwd": prob.plan_f, "plan_bwd": prob.plan_b,
+                      "device_error": err}))
+    return 0 if err == 0 else 1
 
 
 def main(argv=None):
@@ -571,8 +699,13 @@ def main(argv=None):
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--nondeterministic", action="store_true")
-    ap.add_argument("--dw-fp32", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--dw-bf16", action="store_true", help="BF16 dw (default: FP32 dw)")
+    ap.add_argument("--flush", action="store_true",
+                    help="flush L2 before every replay even when the inputs exceed L2")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the per-operation times of the other large workloads")
+    ap.add_argument("--per-config-steps", type=int, default=50)
+    ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-cpu-all-cores", dest="cpu_all_cores", action="store_false",
@@ -581,10 +714,17 @@ def main(argv=None):
                     help="also time an empty graph and torch elementwise kernels the same way")
     ap.add_argument("--ref-seconds", type=float, default=60.0,
                     help="target duration of the reference (oracle) arm")
+    ap.add_argument("--tune", action="append", default=[], metavar="KNOB=VALUE",
+                    help="a gnorm_tuning knob for this run (repeatable; recorded in config)")
+    ap.add_argument("--profile-op", choices=("fwd", "bwd", "ckpt"),
+                    help="run only this operation --reps times and exit (for ncu captures)")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     wl = WORKLOADS[args.workload]
+    if args.profile_op:
+        return run_profile(args, wl)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

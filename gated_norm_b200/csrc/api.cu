@@ -73,6 +73,19 @@ int device_info(DeviceInfo* out) {
   return GNORM_OK;
 }
 
+}  // namespace
+
+// The current device's error word (device address), for entry points in other files.
+int device_error_word(unsigned** out) {
+  DeviceInfo d;
+  const int st = device_info(&d);
+  if (st != GNORM_OK) return st;
+  *out = d.err_word;
+  return GNORM_OK;
+}
+
+namespace {
+
 // A memory region an argument covers: a plain byte span, or a BF16 [rows, cols] matrix
 // with row stride `ld` elements.
 struct Region {

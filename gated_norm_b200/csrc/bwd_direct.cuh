@@ -98,9 +98,9 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectBwdCtasPerSm)
         ue[i] = mul2(mul2(dyp[i], wp[i]), silu);              // dy w s
         dot2 = fma2(ue[i], xhat, dot2);
         if (valid[u]) dwacc[i] = fma2(t, silu, dwacc[i]);
-        // sigmoid' (1 + g (1 - sigmoid)) written as (1 + g) - silu
-        const float2 dsilu = fma2(silu, splat2(-1.0f), add2(gp[i], splat2(1.0f)));
-        dgp[i] = mul2(mul2(mul2(t, wp[i]), sgm), dsilu);
+        // sigmoid' = sigmoid (1 + g (1 - sigmoid))
+        const float2 bracket = gate_grad_bracket(gp[i], sgm);
+        dgp[i] = mul2(mul2(mul2(t, wp[i]), sgm), bracket);
       }
       if (valid[u] && cval)
         *(reinterpret_cast<uint4*>(a.dg + row[u] * a.lddg) + lr) = pairs_to_bf16x8(dgp);

@@ -321,9 +321,9 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
             u[k][i] = ue;
             dot2 = fma2(ue, xhat, dot2);
             if (valid) dwacc[k][i] = fma2(t, silu, dwacc[k][i]);
-            // sigmoid' (1 + g (1 - sigmoid)) written as (1 + g) - silu
-            const float2 dsilu = fma2(silu, splat2(-1.0f), add2(gp[i], splat2(1.0f)));
-            dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), dsilu);
+            // sigmoid' = sigmoid (1 + g (1 - sigmoid))
+            const float2 bracket = gate_grad_bracket(gp[i], sgm);
+            dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), bracket);
           }
           if (valid)
             *reinterpret_cast<uint4*>(a.dg + grow * a.lddg + c * 8) = pairs_to_bf16x8(dgp);

@@ -216,6 +216,15 @@ __device__ __forceinline__ float2 sigmoid2(float2 t) {
   return make_float2(rcp_approx(d.x), rcp_approx(d.y));
 }
 
+// The bracket of the gate's derivative, 1 + g (1 - sigmoid(g)), from the pair's sigmoid:
+// 1 - sigmoid, then one fused multiply-add.  (Written as (1 + g) - g sigmoid(g) it would
+// lose the 1 once g >= 2^24, where 1 + g rounds to g in FP32 and sigmoid(g) is exactly 1;
+// this form keeps it, and gives NaN for g = +inf as the definition does.)
+__device__ __forceinline__ float2 gate_grad_bracket(float2 g, float2 sgm) {
+  const float2 one = splat2(1.0f);
+  return fma2(g, fma2(sgm, splat2(-1.0f), one), one);
+}
+
 // Sum over the `TPR` consecutive threads that share a row.  TPR <= 32: butterfly
 // shuffles inside the warp (every lane of the warp must call).  TPR > 32: butterfly per
 // warp, then the warps of the row exchange partials through shared-memory slots guarded

@@ -19,6 +19,10 @@ cudaError_t launch_bwd(const gnorm_plan& p, const BwdArgs& a, cudaStream_t strea
 cudaError_t launch_dw_reduce(const float* partial, int P, int N, void* dw, int dw_fp32,
                              unsigned long long* work_counter, cudaStream_t stream, bool pdl);
 
+// Device address of the current device's error word (the one gnorm_device_error reads);
+// every kernel's bounded waits report there.  Returns a gnorm_status.
+int device_error_word(unsigned** out);
+
 // Raises a kernel's dynamic shared-memory limit once per (device, kernel).
 inline cudaError_t ensure_smem_limit(const void* kernel, int bytes) {
   static std::mutex mu;

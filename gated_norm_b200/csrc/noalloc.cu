@@ -11,7 +11,8 @@
 // In host code the array's name is only a host-side stand-in, not a device address, so
 // its device address is looked up once per device with cudaGetSymbolAddress (with that
 // device current) and passed to the kernels.  Every call shares the array; the counters
-// that must start at zero are cleared on the stream before each launch.
+// that must start at zero are cleared on the stream before each launch.  A bounded wait that
+// gives up reports through the library's device error word, read by gnorm_device_error.
 #include <cuda_runtime.h>
 
 #include <cmath>
@@ -29,7 +30,6 @@ namespace {
 
 constexpr size_t kStaticScratchBytes = size_t(4) << 20;  // 4 MiB per device
 constexpr int kMaxStaticDevices = 64;
-constexpr int kStaticErrWordOffset = 128;  // inside the cleared header
 
 static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
 
@@ -113,7 +113,14 @@ extern "C" int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, c
   if (st != GNORM_OK) return st;
   if (workspace_bytes_for(plan, N) > kStaticScratchBytes) return GNORM_ERR_UNSUPPORTED;
 
-  // The schedule counter, the completion ticket and the error word start at zero.
+  // A bounded wait that gives up inside these kernels sets its bit in the library's device
+  // error word (itself a static device symbol), so gnorm_device_error reports it as it does
+  // for every other entry point.
+  unsigned* err_word = nullptr;
+  st = device_error_word(&err_word);
+  if (st != GNORM_OK) return st;
+
+  // The schedule counter and the completion ticket start at zero.
   if (cudaMemsetAsync(sc.ptr, 0, kWorkspaceHeader, s) != cudaSuccess) return GNORM_ERR_CUDA;
 
   BwdArgs a;
@@ -141,7 +148,7 @@ extern "C" int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, c
   a.dw_fp32 = dw_fp32 ? 1 : 0;
   a.prefetch = 0;
   a.l2_prefetch = plan.l2_prefetch;
-  a.err = reinterpret_cast<unsigned*>(sc.ptr + kStaticErrWordOffset);
+  a.err = err_word;
   const bool pdl = get_tuning().disable_pdl == 0;
   if (launch_bwd(plan, a, s, pdl) != cudaSuccess) return GNORM_ERR_CUDA;
   if (!plan.fused_reduce &&

@@ -70,7 +70,16 @@ def gnorm_plan_query(kind: int, M: int, N: int, deterministic: bool, num_sms: in
 
 
 def gnorm_device_error(reset: bool = False) -> int:
-    return int(lib.gnorm_device_error(int(bool(reset))))
+    """The device error word (nonzero: a bounded wait inside a kernel gave up).  A call that
+    gave up may leave its workspace header nonzero, so the workspaces this module caches are
+    zeroed again whenever the word is nonzero; workspaces passed in by the caller are the
+    caller's to zero (include/gnorm.h, gnorm_bwd)."""
+    word = int(lib.gnorm_device_error(int(bool(reset))))
+    if word > 0:
+        with _ws_lock:
+            for buf in _ws_cache.values():
+                buf[:256].zero_()
+    return word
 
 
 def gnorm_selftest_wait_timeout(timeout_us: int = 20000) -> int:

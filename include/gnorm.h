@@ -96,8 +96,11 @@ GNORM_API int gnorm_fwd(const void* x, const void* g, const void* w, float eps,
  *
  * workspace: device scratch of at least gnorm_bwd_workspace_bytes(M, N, deterministic)
  *   bytes, GNORM_WORKSPACE_ALIGN-aligned.  Its first GNORM_WORKSPACE_ALIGN bytes must be
- *   zero before the first call (e.g. cudaMemset once after allocation); every call leaves
- *   them zero again.  Concurrent calls must not share a workspace.
+ *   zero before the first call (e.g. cudaMemset once after allocation); every call that
+ *   completes normally leaves them zero again.  A call whose bounded wait gave up (a nonzero
+ *   gnorm_device_error) may return before it restores them, and its outputs are then
+ *   undefined: zero the first GNORM_WORKSPACE_ALIGN bytes again before reusing the
+ *   workspace.  Concurrent calls must not share a workspace.
  */
 GNORM_API int gnorm_bwd(const void* dy, const void* x, const void* g, const void* w, const float* rstd,
               void* dx, void* dg, void* dw, int dw_fp32, int deterministic,
@@ -119,7 +122,8 @@ GNORM_API int gnorm_bwd(const void* dy, const void* x, const void* g, const void
  * capture.  Every call clears the array's 256-byte counter header on `stream` before its
  * kernels start; all calls share the array, so calls that overlap on the GPU (other
  * streams, other threads) race and must be serialised by the caller.  A wait timeout inside
- * these kernels is recorded in the array's header, not in gnorm_device_error's word.
+ * these kernels sets its bit in the device error word that gnorm_device_error reads, as for
+ * every other entry point; the next call clears the array's header again in any case.
  */
 GNORM_API int gnorm_bwd_noalloc(const void* dy, const void* x, const void* g, const void* w,
                                 const float* rstd, void* dx, void* dg, void* dw, int dw_fp32,

@@ -364,3 +364,11 @@ def test_header_is_c_and_links_from_c(tmp_path):
     assert int(fields["ws"]) == gn.gnorm_bwd_workspace_bytes_for(368640, 128, True, 148)
     assert int(fields["null"]) == GNORM_ERR_NULL and int(fields["shape"]) == GNORM_ERR_SHAPE
     assert "sm_100a" in out
+
+
+def test_header_states_the_workspace_rule_after_a_timeout():
+    """A call whose bounded wait gave up may leave the workspace header nonzero; the header
+    tells the caller to zero it again before reuse."""
+    text = open(os.path.join(ROOT, "include", "gnorm.h")).read()
+    assert "zero the first GNORM_WORKSPACE_ALIGN bytes again" in text
+    assert "every call that\n *   completes normally leaves them zero again" in text

@@ -47,3 +47,35 @@ def test_single_rank_combine_is_identity():
     out = gn.gnorm_dw_reduce(dw_local.view(1, -1))
     torch.cuda.synchronize()
     assert torch.equal(out, dw_local)
+
+
+def test_allreduce_dw_single_rank_process_group():
+    """gated_norm_b200.dp.allreduce_dw end to end in a world-size-1 NCCL process group: the
+    gather returns this rank's row and the fixed-order sum is bitwise gnorm_dw_reduce of it
+    (and, for one FP32 row, the row itself)."""
+    import socket
+
+    import torch.distributed as dist
+
+    from gated_norm_b200.dp import allreduce_dw
+    from gpu_util import Case
+
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    case = Case(4099, 256, seed=3)
+    _, rstd = gn.gnorm_fwd(case.x, case.g, case.w, case.eps)
+    _, _, dw_local = gn.gnorm_bwd(case.dy, case.x, case.g, case.w, rstd, dw_fp32=True)
+    torch.cuda.synchronize()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0,
+                            world_size=1, device_id=torch.device("cuda", 0))
+    try:
+        for fp32 in (True, False):
+            got = allreduce_dw(dw_local, dw_fp32=fp32)
+            ref = gn.gnorm_dw_reduce(dw_local.view(1, -1), dw_fp32=fp32)
+            torch.cuda.synchronize()
+            assert torch.equal(got.view(torch.uint8), ref.view(torch.uint8)), fp32
+        assert torch.equal(allreduce_dw(dw_local), dw_local)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()

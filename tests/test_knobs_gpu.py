@@ -11,8 +11,9 @@ import itertools
 import pytest
 import torch
 
-from gpu_util import Case, dev_to_f64
-from tolerance import dw_fp32_check
+from gpu_util import Case, dev_to_f64, sample_rows
+from synthetic import WORKLOADS
+from tolerance import bf16_check, dw_fp32_check, rstd_check
 
 pytestmark = pytest.mark.gpu
 
@@ -106,4 +107,49 @@ def test_direct_and_staged_kernels_agree(M, N, w_fp32, strided):
     for out in bwd:
         rep = dw_fp32_check(dev_to_f64(out[2]), dw_ref)
         assert rep["ok"], rep
+    assert gn.gnorm_device_error(reset=True) == 0
+
+
+@pytest.mark.parametrize("det", [True, False])
+def test_l2_prefetch_reaches_its_copies(det):
+    """The L2 prefetch (flashinfer PR #8701, commit message: thread 0 warms L2 with the CTA's
+    next row block) only issues copies when a CTA holds more row blocks than its ring: at
+    368640 x 128 the staged forward has 2 stages of ~96 rows for ~13 blocks per CTA and the
+    backward 3 stages for ~9, so most blocks prefetch the one a ring further on.  Results must
+    not change at all (a prefetch writes no register and no memory) and must match the
+    oracle on sampled rows and in dw."""
+    wl = WORKLOADS["long_368640x128"]
+    case = Case(wl.M, wl.N, seed=wl.seed, g_std=wl.g_std)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    outs = []
+    try:
+        for mode in (2, 1):
+            gn.gnorm_set_tuning(l2_prefetch=mode)
+            pf, pb = gn.gnorm_plan_query(0, wl.M, wl.N, det, sms), gn.gnorm_plan_query(1, wl.M, wl.N, det, sms)
+            assert pf["l2_prefetch"] == (mode == 1) and pb["l2_prefetch"] == (mode == 1)
+            assert not pf["direct_loads"] and not pb["direct_loads"]
+            # more blocks per CTA than ring stages: the prefetch branch is taken
+            assert pf["num_blocks"] > pf["grid"] * pf["stages"]
+            assert pb["num_blocks"] > pb["grid"] * pb["stages"]
+            y, rstd = gn.gnorm_fwd(case.x, case.g, case.w, case.eps)
+            dx, dg, dw = gn.gnorm_bwd(case.dy, case.x, case.g, case.w, rstd, dw_fp32=True,
+                                      deterministic=det)
+            outs.append((y, rstd, dx, dg, dw))
+        torch.cuda.synchronize()
+    finally:
+        gn.gnorm_set_tuning()
+    for a, b, name in zip(outs[0][:4], outs[1][:4], ("y", "rstd", "dx", "dg")):
+        assert torch.equal(a, b), name
+    if det:
+        assert torch.equal(outs[0][4], outs[1][4])
+    y, rstd, dx, dg, dw = outs[1]
+    rows = sample_rows(wl.M, n_random=4096)
+    ry, rr, rdx, rdg = case.oracle_rows(rows)
+    idx = torch.from_numpy(rows).cuda()
+    for got, ref, name, chk in ((y, ry, "y", bf16_check), (rstd, rr, "rstd", rstd_check),
+                                (dx, rdx, "dx", bf16_check), (dg, rdg, "dg", bf16_check)):
+        rep = chk(dev_to_f64(got[idx]), ref)
+        assert rep["ok"], (name, rep)
+    rep = dw_fp32_check(dev_to_f64(dw), case.oracle_dw())
+    assert rep["ok"], rep
     assert gn.gnorm_device_error(reset=True) == 0

@@ -53,6 +53,40 @@ def test_degenerate_rows():
     assert np.isnan(rn[0]) and np.all(np.isnan(yn))
 
 
+def test_infinities_and_huge_gates_follow_ieee_and_the_library():
+    """Non-finite inputs follow IEEE arithmetic through the definition, as the library
+    routines of the comparators' form do (torch sigmoid / silu / rms_norm in FP64): silu(+inf)
+    = +inf, silu(-inf) = -inf * 0 = NaN; an infinite x gives r = 0, so that row's y is 0
+    except NaN at the infinite element.  For a huge finite gate (sigmoid rounds to exactly 1
+    in FP64) the gate derivative's bracket 1 + g (1 - sigmoid) is exactly 1, so
+    dg = dy * xhat * w (closed form)."""
+    import torch
+
+    g = np.array([-np.inf, np.inf, -1e30, 1e30, 3e7, np.nan])
+    tg = torch.tensor(g, dtype=torch.float64)
+    with np.errstate(invalid="ignore"):
+        np.testing.assert_array_equal(oracle.silu(g), torch.nn.functional.silu(tg).numpy())
+    np.testing.assert_array_equal(oracle.sigmoid(g), torch.sigmoid(tg).numpy())
+    N = 8
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((2, N))
+    x[1, 3] = np.inf
+    gg = rng.standard_normal((2, N))
+    w = 1 + 0.1 * rng.standard_normal(N)
+    with np.errstate(invalid="ignore"):
+        y, r = oracle.fwd(x, gg, w, 1e-6)
+    assert r[1] == 0.0 and np.isnan(y[1, 3])
+    assert np.all(y[1, np.arange(N) != 3] == 0.0)
+    ty = torch.nn.functional.rms_norm(torch.tensor(x[:1]), (N,), eps=1e-6).numpy()
+    np.testing.assert_allclose(y[0], (ty * w * gg[:1] * scipy.special.expit(gg[:1]))[0],
+                               rtol=1e-13)
+    big = np.full((1, N), 3e7)
+    dy = rng.standard_normal((1, N))
+    _, rb = oracle.fwd(x[:1], big, w, 1e-6)
+    _, dg, _ = oracle.bwd(dy, x[:1], big, w, rb)
+    np.testing.assert_array_equal(dg, dy * (x[:1] * rb[:, None]) * w[None, :])
+
+
 def test_ckpt_step_is_two_forwards_then_backward():
     rng = np.random.default_rng(12)
     x, g, dy = (rng.standard_normal((3, 8)) for _ in range(3))

@@ -43,3 +43,45 @@ def test_subnormal_results_may_flush_to_zero():
     ref = np.array([[1e-40, -3e-39, 0.0]])
     assert bf16_check(np.zeros_like(ref), ref)["ok"]
     assert not bf16_check(np.array([[1e-37, 0.0, 0.0]]), ref)["ok"]
+
+
+def test_nonfinite_reference_must_be_matched():
+    ref = np.array([[1.0, np.nan, np.inf, -np.inf, 2.0]])
+    gpu = ref.copy()
+    assert bf16_check(gpu, ref)["ok"]
+    # a NaN turned into a number, an infinity of the wrong sign, a finite value for an
+    # infinity, and an infinity or NaN where the oracle is finite are all failures
+    for j, v in ((1, 0.0), (2, -np.inf), (3, 3e38), (0, np.inf), (4, np.nan)):
+        g = ref.copy()
+        g[0, j] = v
+        assert not bf16_check(g, ref)["ok"], (j, v)
+        assert not dw_fp32_check(g[0], ref[0])["ok"], (j, v)
+    assert dw_fp32_check(ref[0], ref[0])["ok"]
+
+
+def test_nan_elsewhere_in_a_row_does_not_void_the_rest():
+    rng = np.random.default_rng(3)
+    ref = rng.standard_normal((4, 32))
+    ref[1, 5] = np.nan
+    ref[2, 7] = np.inf
+    gpu = ref.copy()
+    assert bf16_check(gpu, ref)["ok"]
+    gpu[1, 6] += 0.5  # a wrong finite element in the row that holds the NaN
+    rep = bf16_check(gpu, ref)
+    assert not rep["ok"] and rep["first_bad"] == [1, 6]
+    gpu = ref.copy()
+    gpu[2, 0] *= 1.2  # and in the row that holds the infinity
+    assert not bf16_check(gpu, ref)["ok"]
+
+
+def test_rstd_nonfinite():
+    ref = np.array([1.0, np.nan, 3.0])
+    assert rstd_check(ref.copy(), ref)["ok"]
+    assert not rstd_check(np.array([1.0, 1.0, 3.0]), ref)["ok"]
+    assert not rstd_check(np.array([1.0, np.nan, np.inf]), ref)["ok"]
+
+
+def test_rstd_zero_reference_needs_zero():
+    ref = np.array([0.0, 2.0])
+    assert rstd_check(np.array([0.0, 2.0]), ref)["ok"]
+    assert not rstd_check(np.array([1e-30, 2.0]), ref)["ok"]
