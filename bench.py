@@ -719,10 +719,15 @@ def main(argv=None):
     ap.add_argument("--profile-op", choices=("fwd", "bwd", "ckpt"),
                     help="run only this operation --reps times and exit (for ncu captures)")
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--rows", type=int, default=0,
+                    help="override the workload's row count (same distributions; for "
+                         "smaller profiling cases)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     wl = WORKLOADS[args.workload]
+    if args.rows:
+        wl = wl.scaled(args.rows)
     if args.profile_op:
         return run_profile(args, wl)
     if args.impl == "reference":

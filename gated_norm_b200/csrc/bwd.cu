@@ -48,6 +48,11 @@ cudaError_t launch_bwd(const gnorm_plan& p, const BwdArgs& a, cudaStream_t strea
     case 4 * 8 + 1: return launch_bwd_geometry<4, 1>(p, a, stream, pdl);
     case 8 * 8 + 1: return launch_bwd_geometry<8, 1>(p, a, stream, pdl);
     case 16 * 8 + 1: return launch_bwd_geometry<16, 1>(p, a, stream, pdl);
+    case 4 * 8 + 4: return launch_bwd_geometry<4, 4>(p, a, stream, pdl);
+    case 8 * 8 + 2: return launch_bwd_geometry<8, 2>(p, a, stream, pdl);
+    case 8 * 8 + 4: return launch_bwd_geometry<8, 4>(p, a, stream, pdl);
+    case 16 * 8 + 2: return launch_bwd_geometry<16, 2>(p, a, stream, pdl);
+    case 16 * 8 + 4: return launch_bwd_geometry<16, 4>(p, a, stream, pdl);
     case 32 * 8 + 1: return launch_bwd_geometry<32, 1>(p, a, stream, pdl);
     case 32 * 8 + 2: return launch_bwd_geometry<32, 2>(p, a, stream, pdl);
     case 32 * 8 + 4: return launch_bwd_geometry<32, 4>(p, a, stream, pdl);

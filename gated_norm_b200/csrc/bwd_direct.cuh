@@ -84,11 +84,10 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectBwdCtasPerSm)
     for (int u = 0; u < kU; ++u) {
       const float r = rv[u];
       const float2 r2 = splat2(r);
-      float2 dyp[4], xp[4], gp[4], dgp[4], ue[4];
+      float2 dyp[4], xp[4], gp[4], dgp[4], ue[4], xh[4];
       bf16x8_to_pairs(dyv[u], dyp);
       bf16x8_to_pairs(xv[u], xp);
       bf16x8_to_pairs(gv[u], gp);
-      float2 dot2 = splat2(0.f);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float2 xhat = mul2(xp[i], r2);
@@ -96,7 +95,7 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectBwdCtasPerSm)
         const float2 silu = mul2(gp[i], sgm);
         const float2 t = mul2(dyp[i], xhat);                 // dy xhat
         ue[i] = mul2(mul2(dyp[i], wp[i]), silu);              // dy w s
-        dot2 = fma2(ue[i], xhat, dot2);
+        xh[i] = xhat;
         if (valid[u]) dwacc[i] = fma2(t, silu, dwacc[i]);
         // sigmoid' = sigmoid (1 + g (1 - sigmoid))
         const float2 bracket = gate_grad_bracket(gp[i], sgm);
@@ -104,7 +103,7 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectBwdCtasPerSm)
       }
       if (valid[u] && cval)
         *(reinterpret_cast<uint4*>(a.dg + row[u] * a.lddg) + lr) = pairs_to_bf16x8(dgp);
-      const float dot = row_sum<TPR>(dot2.x + dot2.y, nullptr, group, lr, 0);
+      const float dot = row_sum<TPR>(chunk_dot(ue, xh), nullptr, group, lr, 0);
       const float2 nrc2 = splat2(-(r * (dot * a.inv_n)));
       float2 dxp[4];
 #pragma unroll

@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
   const int ctid = threadIdx.x - 32;
   const int group = ctid / TPR;
   const int lr = ctid - group * TPR;
+  const int warp_group0 = (ctid & ~31) / TPR;  // first row slot of this warp
   const int n8 = N >> 3;
 
   float2 wp[CPT][4];     // this thread's weights, as FP32 pairs
@@ -291,6 +292,9 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
     const float* srs = reinterpret_cast<const float*>(sg + tensor_bytes);
 
     for (int rb = 0; rb < rows; rb += kGroups) {
+      // A warp whose rows are all past the block's end skips the pass (a warp never spans
+      // two row groups' barriers, so this is uniform per warp and per row group).
+      if (rb + warp_group0 >= rows) break;
       const int row = rb + group;
       const bool valid = row < rows;
       const int srow = valid ? row : 0;
@@ -301,13 +305,14 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
 
       // pass 1: recompute xhat and the gate; dg; row dot product; dw accumulators
       float2 u[CPT][4];
-      float2 dot2 = splat2(0.f);
+      float part[CPT];
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
+        part[k] = 0.f;
         if (cval[k]) {
           const int c = k * TPR + lr;
           const size_t off = roff + static_cast<size_t>(c) * 16;
-          float2 dyp[4], xp[4], gp[4], dgp[4];
+          float2 dyp[4], xp[4], gp[4], dgp[4], xh[4];
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sg + off), gp);
@@ -319,17 +324,18 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
             const float2 t = mul2(dyp[i], xhat);                    // dy xhat
             const float2 ue = mul2(mul2(dyp[i], wp[k][i]), silu);    // dy w s
             u[k][i] = ue;
-            dot2 = fma2(ue, xhat, dot2);
+            xh[i] = xhat;
             if (valid) dwacc[k][i] = fma2(t, silu, dwacc[k][i]);
             // sigmoid' = sigmoid (1 + g (1 - sigmoid))
             const float2 bracket = gate_grad_bracket(gp[i], sgm);
             dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), bracket);
           }
+          part[k] = chunk_dot(u[k], xh);  // this chunk's share of sum(u xhat)
           if (valid)
             *reinterpret_cast<uint4*>(a.dg + grow * a.lddg + c * 8) = pairs_to_bf16x8(dgp);
         }
       }
-      const float dot = row_sum<TPR>(dot2.x + dot2.y, red_slots, group, lr, slot);
+      const float dot = row_sum<TPR>(combine_chunks<CPT>(part), red_slots, group, lr, slot);
       slot ^= 1;
       const float2 nrc2 = splat2(-(r * (dot * a.inv_n)));
 

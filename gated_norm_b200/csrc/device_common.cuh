@@ -57,25 +57,47 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
   return done != 0;
 }
 
+// The same test with a suspend-time hint: while the phase is incomplete the thread may sleep
+// in hardware (woken when the phase completes, or after about `hint_ns`) instead of spinning,
+// so waiting warps do not take issue slots from the warps that compute.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar_addr, uint32_t parity,
+                                                      uint32_t hint_ns) {
+  uint32_t done;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(done)
+      : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return done != 0;
+}
+
+// Suspend hint of the pipeline waits (ns): long against a stage's arrival, short against
+// the waits' time limit, which is checked after every try.
+constexpr uint32_t kWaitSuspendNs = 20000;
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
 
-// Waits until the barrier phase with the given parity has completed.  Gives up after
-// kWaitLimitNs (or 2^24 polling rounds, whichever comes first), sets `err_bit` in the
-// device error word and returns false; the caller then stops its loop and exits.
+// Waits until the barrier phase with the given parity has completed, sleeping between tries
+// (suspend hint).  Gives up after `limit_ns` (or 2^24 tries, whichever comes first), sets
+// `err_bit` in the device error word and returns false; the caller then stops its loop and
+// exits.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsigned* err_word,
                                           unsigned err_bit,
                                           unsigned long long limit_ns = kWaitLimitNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
+  const uint32_t hint = limit_ns < 8ull * kWaitSuspendNs
+                            ? static_cast<uint32_t>(limit_ns / 8) + 1u
+                            : kWaitSuspendNs;
   for (uint32_t round = 0; round < (1u << 24); ++round) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(a, parity)) return true;
+    if (mbar_try_wait_suspend(a, parity, hint)) return true;
     if (globaltimer_ns() - t0 > limit_ns) break;
   }
   atomicOr(err_word, err_bit);
@@ -223,6 +245,30 @@ __device__ __forceinline__ float2 sigmoid2(float2 t) {
 __device__ __forceinline__ float2 gate_grad_bracket(float2 g, float2 sgm) {
   const float2 one = splat2(1.0f);
   return fma2(g, fma2(sgm, splat2(-1.0f), one), one);
+}
+
+// Row reductions in an order that does not depend on the row geometry.  Each 16-byte chunk
+// (8 values, 4 pairs) reduces to one partial in a fixed order; a thread's CPT chunks
+// (chunk indices lr, lr + TPR, ..., lr + (CPT - 1) TPR) are then combined by halving, which
+// is exactly what the first log2(CPT) levels of a butterfly over CPT x TPR one-chunk threads
+// would add.  So a geometry with CPT chunks per thread and one with a single chunk per
+// thread produce bitwise the same row sums, and the direct-load and staged kernels the
+// same results.
+__device__ __forceinline__ float chunk_dot(const float2 a[4], const float2 b[4]) {
+  float2 s = mul2(a[0], b[0]);
+#pragma unroll
+  for (int i = 1; i < 4; ++i) s = fma2(a[i], b[i], s);
+  return s.x + s.y;
+}
+
+template <int CPT>
+__device__ __forceinline__ float combine_chunks(float part[CPT]) {
+#pragma unroll
+  for (int h = CPT / 2; h >= 1; h /= 2) {
+#pragma unroll
+    for (int k = 0; k < h; ++k) part[k] = part[k] + part[k + h];
+  }
+  return part[0];
 }
 
 // Sum over the `TPR` consecutive threads that share a row.  TPR <= 32: butterfly

@@ -69,10 +69,7 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectCtasPerSm)
     for (int u = 0; u < kU; ++u) {
       float2 xp[4];
       bf16x8_to_pairs(xv[u], xp);
-      float2 ss2 = splat2(0.f);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) ss2 = fma2(xp[i], xp[i], ss2);
-      const float ss = row_sum<TPR>(ss2.x + ss2.y, nullptr, group, lr, 0);
+      const float ss = row_sum<TPR>(chunk_dot(xp, xp), nullptr, group, lr, 0);
       r[u] = rsqrtf(fmaf(ss, a.inv_n, a.eps));
       if (valid[u] && lr == 0) a.rstd[row[u]] = r[u];
     }

@@ -129,6 +129,7 @@ __global__ void __launch_bounds__(consumer_threads_for(0, TPR, CPT) + 32, max_ct
   const int ctid = threadIdx.x - 32;
   const int group = ctid / TPR;         // row slot inside a pass over the stage
   const int lr = ctid - group * TPR;    // thread index inside the row
+  const int warp_group0 = (ctid & ~31) / TPR;  // first row slot of this warp
   const int n8 = N >> 3;                // 16-byte chunks per row
 
   float2 wp[CPT][4];  // this thread's weights, as FP32 pairs
@@ -156,25 +157,29 @@ __global__ void __launch_bounds__(consumer_threads_for(0, TPR, CPT) + 32, max_ct
     const uint8_t* sg = sx + tensor_bytes;
 
     for (int rb = 0; rb < rows; rb += kGroups) {
+      // A warp whose rows are all past the block's end skips the pass (a warp never spans
+      // two row groups' barriers, so this is uniform per warp and per row group).
+      if (rb + warp_group0 >= rows) break;
       const int row = rb + group;
       const bool valid = row < rows;
       const int srow = valid ? row : 0;  // keep shared-memory reads inside the stage
       const size_t roff = static_cast<size_t>(srow) * N * 2;
 
-      // pass 1: sum of squares of the row (two interleaved FP32 partial sums per thread)
+      // pass 1: sum of squares of the row (one partial per chunk, combined in the order
+      // every row geometry shares)
       uint4 xv[CPT];
-      float2 ss2 = splat2(0.f);
+      float part[CPT];
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
+        part[k] = 0.f;
         if (cval[k]) {
           xv[k] = *reinterpret_cast<const uint4*>(sx + roff + (k * TPR + lr) * 16);
           float2 xp[4];
           bf16x8_to_pairs(xv[k], xp);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) ss2 = fma2(xp[i], xp[i], ss2);
+          part[k] = chunk_dot(xp, xp);
         }
       }
-      const float ss = row_sum<TPR>(ss2.x + ss2.y, red_slots, group, lr, slot);
+      const float ss = row_sum<TPR>(combine_chunks<CPT>(part), red_slots, group, lr, slot);
       slot ^= 1;
       const float r = rsqrtf(fmaf(ss, a.inv_n, a.eps));
       const long long grow = r0 + row;

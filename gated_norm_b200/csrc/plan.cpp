@@ -33,7 +33,8 @@ TuningKnobs get_tuning() { return g_knobs; }
 bool geometry_compiled(int kind, int tpr, int cpt) {
   static const int kBoth[][2] = {{4, 1},   {8, 1},   {16, 1},  {32, 1},  {32, 2},
                                  {32, 4},  {64, 2},  {64, 4},  {128, 2}, {128, 4},
-                                 {256, 2}, {256, 4}, {512, 4}};
+                                 {256, 2}, {256, 4}, {512, 4}, {4, 4},   {8, 2},
+                                 {8, 4},   {16, 2},  {16, 4}};
   static const int kFwdOnly[][2] = {{64, 8}};
   for (const auto& g : kBoth)
     if (g[0] == tpr && g[1] == cpt) return true;
@@ -43,18 +44,32 @@ bool geometry_compiled(int kind, int tpr, int cpt) {
   return false;
 }
 
+// Staged kernels: two 16-byte chunks per thread from N > 64 on (measured on B200, same box:
+// 262144 x 256 forward 69.8 -> 66.0 us and backward 116.9 -> 106.9 us with 16 x 2 instead of
+// 32 x 1; 368640 x 128 forward 48.7 -> 47.8 us with 8 x 2 instead of 16 x 1, backward equal).
 RowGeometry geometry_for(int64_t N) {
   const int64_t n8 = N / 8;  // 16-byte chunks per row
   if (n8 <= 4) return {4, 1};
   if (n8 <= 8) return {8, 1};
-  if (n8 <= 16) return {16, 1};
-  if (n8 <= 32) return {32, 1};
+  if (n8 <= 16) return {8, 2};
+  if (n8 <= 32) return {16, 2};
   if (n8 <= 64) return {32, 2};
   if (n8 <= 128) return {64, 2};
   if (n8 <= 256) return {128, 2};
   if (n8 <= 512) return {256, 2};
   if (n8 <= 1024) return {256, 4};
   return {512, 4};
+}
+
+// Direct-load kernels (rows of N <= 256): one 16-byte chunk per thread, so a row is at most
+// one warp; {0, 0} for wider rows.
+RowGeometry direct_geometry_for(int64_t N) {
+  const int64_t n8 = N / 8;
+  if (n8 <= 4) return {4, 1};
+  if (n8 <= 8) return {8, 1};
+  if (n8 <= 16) return {16, 1};
+  if (n8 <= 32) return {32, 1};
+  return {0, 0};
 }
 
 static int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
@@ -69,11 +84,14 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   if (smem_per_block <= 0) smem_per_block = kB200SmemPerBlock;
 
   RowGeometry geo = geometry_for(N);
+  RowGeometry dgeo = direct_geometry_for(N);
   if (g_knobs.threads_per_row > 0 && g_knobs.chunks_per_thread > 0) {
     geo = {g_knobs.threads_per_row, g_knobs.chunks_per_thread};
     if (!geometry_compiled(kind, geo.threads_per_row, geo.chunks_per_thread) ||
         static_cast<int64_t>(geo.threads_per_row) * geo.chunks_per_thread * 8 < N)
       return GNORM_ERR_UNSUPPORTED;
+    // a forced geometry applies to the direct-load kernels too, where they can run it
+    dgeo = (geo.chunks_per_thread == 1 && geo.threads_per_row <= 32) ? geo : RowGeometry{0, 0};
   }
   const int nct = consumer_threads_for(kind, geo.threads_per_row, geo.chunks_per_thread);
   const int groups = nct / geo.threads_per_row;
@@ -85,10 +103,11 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   const bool latency_tier = kind == 0 && rows_per_sm * row_bytes < kFwdLatencyTierBytes;
   // Forward of narrow rows in the latency tier (or always / never, by knob): rows loaded
   // straight into registers, no shared-memory stages.
-  const bool direct_capable = kind == 0 && geo.chunks_per_thread == 1 && geo.threads_per_row <= 32;
+  const bool direct_capable = kind == 0 && dgeo.threads_per_row > 0;
   const bool direct = direct_capable && (g_knobs.fwd_direct == 1 ||
                                          (g_knobs.fwd_direct == 0 && latency_tier));
   if (direct) {
+    geo = dgeo;
     const int64_t rows_per_iter =
         static_cast<int64_t>(kDirectThreads / geo.threads_per_row) * kDirectRows;
     const int ctas = std::min(kDirectCtasPerSm,
@@ -109,9 +128,10 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   }
 
   // Backward of narrow rows with very few rows per SM: straight into registers as well.
-  const bool bwd_capable = kind == 1 && geo.chunks_per_thread == 1 && geo.threads_per_row <= 32;
+  const bool bwd_capable = kind == 1 && dgeo.threads_per_row > 0;
   const bool bwd_tier = rows_per_sm * (3 * N * 2) < kBwdDirectTierBytes;
   if (bwd_capable && (g_knobs.bwd_direct == 1 || (g_knobs.bwd_direct == 0 && bwd_tier))) {
+    geo = dgeo;
     const int64_t rows_per_iter =
         static_cast<int64_t>(kDirectThreads / geo.threads_per_row) * kDirectBwdRows;
     const int ctas = std::min(kDirectBwdCtasPerSm, g_knobs.ctas_per_sm > 0
