@@ -70,7 +70,7 @@ cudaError_t launch_bwd(const gnorm_plan& p, const BwdArgs& a, cudaStream_t strea
 cudaError_t launch_dw_reduce(const float* partial, int P, int N, void* dw, int dw_fp32,
                              unsigned long long* work_counter, cudaStream_t stream, bool pdl) {
   const int col_quads = N / 4;
-  const int grid = (col_quads + 31) / 32;
+  const int grid = (col_quads + kReduceQuads - 1) / kReduceQuads;
   return launch_kernel(dw_reduce_kernel, grid, kReduceThreads, 0, stream, pdl, partial, P, N, dw,
                        dw_fp32, work_counter);
 }

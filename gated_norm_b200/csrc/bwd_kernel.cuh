@@ -16,9 +16,9 @@
 // reduction pass 2 re-reads x and writes dx.  The producer warp also stages the rows' rstd
 // with 4-byte asynchronous copies tracked by the same stage barrier.  At the end each CTA adds its row groups' dw accumulators in a fixed order into one
 // FP32 partial row [P, N] in the workspace.  A second pass sums the P partials in a fixed
-// tree order and writes dw once, rounded to BF16 or kept in FP32: by default a second launch
-// whose CTAs share the columns; optionally (small partials) the backward's last CTA to
-// finish, found with an integer ticket, never a wait.
+// order and writes dw once, rounded to BF16 or kept in FP32: by default a second launch whose
+// CTAs each own a few column quads; optionally (small partials) the backward's last CTA to finish,
+// found with an integer ticket, never a wait.
 #pragma once
 
 #include "args.h"
@@ -102,18 +102,84 @@ __device__ __forceinline__ void reduce_partials(const float* __restrict__ partia
   }
 }
 
-// Second pass over the dw partials (both modes): one 1024-thread CTA per 128 columns, so
-// 32 lanes share the partial rows and each issues all its loads at once for P <= 256.
-// Also clears the dynamic-schedule counter of the workspace (the backward grid has
-// finished by now).
+// Second pass over the dw partials (both modes).  A CTA of kReduceThreads threads owns
+// kReduceQuads column quads (4 columns each); thread t takes quad t % kReduceQuads and row lane
+// t / kReduceQuads (kReduceLanes lanes).  A lane adds partial rows lane, lane + kReduceLanes,
+// ... of its quad in increasing order, all its loads in one batch for P <= 8 kReduceLanes; the
+// lanes of a quad are then combined by a fixed tree: inside the warp by shuffles over its 4 row
+// lanes (xor 8, then xor 16), then across the warps through shared memory, pairwise (offsets
+// 4, 2, 1).  The order depends only on P.  A warp's loads are 4 rows x 128 contiguous bytes.
+// Also clears the dynamic-schedule counter of the workspace (the backward grid has finished
+// by now).
 __global__ void __launch_bounds__(kReduceThreads)
     dw_reduce_kernel(const float* __restrict__ partial, int P, int N, void* dw, int dw_fp32,
                      unsigned long long* work_counter) {
-  __shared__ float4 scratch[kReduceThreads];
+  constexpr int kWarps = kReduceThreads / 32;
+  constexpr int kBatch = 8;
+  __shared__ float4 red[kWarps][kReduceQuads];
   grid_dependency_wait();
   allow_dependent_launch();
-  reduce_partials<false>(partial, P, N, dw, dw_fp32, blockIdx.x * 32, gridDim.x * 32,
-                         threadIdx.x, kReduceThreads, scratch);
+  const int q = threadIdx.x % kReduceQuads;
+  const int rl = threadIdx.x / kReduceQuads;
+  const int warp = threadIdx.x >> 5;
+  const int n4 = N >> 2;
+  const int j4 = blockIdx.x * kReduceQuads + q;
+  const bool valid = j4 < n4;
+  const float4* p4 = reinterpret_cast<const float4*>(partial);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int b0 = rl; b0 < P; b0 += kReduceLanes * kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int b = b0 + kReduceLanes * i;
+      v[i] = (valid && b < P) ? __ldcg(p4 + static_cast<size_t>(b) * n4 + j4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      if (b0 + kReduceLanes * i < P) {
+        acc.x += v[i].x;
+        acc.y += v[i].y;
+        acc.z += v[i].z;
+        acc.w += v[i].w;
+      }
+    }
+  }
+  // the warp's 4 row lanes (lane bits 3 and 4)
+#pragma unroll
+  for (int off = kReduceQuads; off < 32; off <<= 1) {
+    acc.x += __shfl_xor_sync(0xffffffffu, acc.x, off);
+    acc.y += __shfl_xor_sync(0xffffffffu, acc.y, off);
+    acc.z += __shfl_xor_sync(0xffffffffu, acc.z, off);
+    acc.w += __shfl_xor_sync(0xffffffffu, acc.w, off);
+  }
+  if ((threadIdx.x & 31) < kReduceQuads) red[warp][q] = acc;
+  __syncthreads();
+#pragma unroll
+  for (int st = kWarps / 2; st > 0; st >>= 1) {
+    if (threadIdx.x < st * kReduceQuads) {
+      const int w = threadIdx.x / kReduceQuads;
+      float4 m = red[w][q];
+      const float4 o = red[w + st][q];
+      m.x += o.x;
+      m.y += o.y;
+      m.z += o.z;
+      m.w += o.w;
+      red[w][q] = m;
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x < kReduceQuads && valid) {
+    const float4 m = red[0][q];
+    if (dw_fp32) {
+      reinterpret_cast<float4*>(dw)[j4] = m;
+    } else {
+      uint2 h;
+      h.x = pack_bf16x2(m.x, m.y);
+      h.y = pack_bf16x2(m.z, m.w);
+      reinterpret_cast<uint2*>(dw)[j4] = h;
+    }
+  }
   if (work_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0ull;
 }
 

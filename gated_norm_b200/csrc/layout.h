@@ -13,7 +13,10 @@ constexpr int kMaxStages = 16;       // mbarrier pairs reserved in the shared-me
 constexpr int kHeaderBytes = 1024;   // barriers, block ids, flags and reduction slots
 constexpr int kRedSlotOffset = 512;  // float slots for cross-warp row reductions
 constexpr int kWorkspaceHeader = 256;  // workspace bytes before the dw partials
-constexpr int kReduceThreads = 1024;  // dw second pass: 32 partial lanes x 32 column quads
+// dw second pass: a CTA owns kReduceQuads column quads, with kReduceLanes row lanes each
+constexpr int kReduceThreads = 256;
+constexpr int kReduceQuads = 8;
+constexpr int kReduceLanes = kReduceThreads / kReduceQuads;
 
 // Computing threads per CTA for a row geometry: 8 warps; one 16-warp row group for the
 // widest rows; and 16 warps for the backward of narrow rows (<= 16 threads per row, one

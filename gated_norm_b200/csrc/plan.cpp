@@ -44,14 +44,16 @@ bool geometry_compiled(int kind, int tpr, int cpt) {
   return false;
 }
 
-// Staged kernels: two 16-byte chunks per thread from N > 64 on (measured on B200, same box:
-// 262144 x 256 forward 69.8 -> 66.0 us and backward 116.9 -> 106.9 us with 16 x 2 instead of
-// 32 x 1; 368640 x 128 forward 48.7 -> 47.8 us with 8 x 2 instead of 16 x 1, backward equal).
-RowGeometry geometry_for(int64_t N) {
+// Staged kernels: two 16-byte chunks per thread for 128 < N <= 256, and for the forward from
+// N > 64 on (measured on B200, same box, back-to-back graph replays: 262144 x 256 forward
+// 69.8 -> 66.0 us and backward 116.9 -> 106.9 us with 16 x 2 instead of 32 x 1; 368640 x 128
+// forward 48.7 -> 47.8 us with 8 x 2 instead of 16 x 1; the backward of rows of 128 keeps 16 x 1
+// with 16 computing warps: equal at 368640 x 128, 19.8 against 20.5 us at 65536 x 128).
+RowGeometry geometry_for(int kind, int64_t N) {
   const int64_t n8 = N / 8;  // 16-byte chunks per row
   if (n8 <= 4) return {4, 1};
   if (n8 <= 8) return {8, 1};
-  if (n8 <= 16) return {8, 2};
+  if (n8 <= 16) return kind == 0 ? RowGeometry{8, 2} : RowGeometry{16, 1};
   if (n8 <= 32) return {16, 2};
   if (n8 <= 64) return {32, 2};
   if (n8 <= 128) return {64, 2};
@@ -83,7 +85,7 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   if (num_sms <= 0) return GNORM_ERR_ARG;
   if (smem_per_block <= 0) smem_per_block = kB200SmemPerBlock;
 
-  RowGeometry geo = geometry_for(N);
+  RowGeometry geo = geometry_for(kind, N);
   RowGeometry dgeo = direct_geometry_for(N);
   if (g_knobs.threads_per_row > 0 && g_knobs.chunks_per_thread > 0) {
     geo = {g_knobs.threads_per_row, g_knobs.chunks_per_thread};

@@ -57,7 +57,7 @@ TuningKnobs get_tuning();
 // Row geometries with compiled kernels, per kind (0 forward, 1 backward).
 bool geometry_compiled(int kind, int threads_per_row, int chunks_per_thread);
 
-RowGeometry geometry_for(int64_t N);
+RowGeometry geometry_for(int kind, int64_t N);
 int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
               int smem_per_block, gnorm_plan* out);
 size_t workspace_bytes_for(const gnorm_plan& p, int64_t N);
