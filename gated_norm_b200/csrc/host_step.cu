@@ -202,12 +202,21 @@ extern "C" int gnorm_ckpt_step_host(const void* x, const void* g, const void* w,
   }
 
   // Fork: the copies in wait for everything already on the caller's stream.  The
-  // workspace's counters start at zero.
-  if (!ok(cudaMemsetAsync(ws_dev, 0, GNORM_WORKSPACE_ALIGN, s)) || !ok(cudaEventRecord(p->start, s)) ||
-      !ok(cudaStreamWaitEvent(p->in, p->start, 0)) || !ok(cudaStreamWaitEvent(p->out, p->start, 0)))
-    return GNORM_ERR_CUDA;
+  // workspace's counters start at zero.  From here on every return joins the copy streams
+  // back into the caller's stream (best effort on a failing runtime), so even a call that
+  // fails part way stays ordered on `stream`; its outputs are then undefined.
+  auto fail = [&](int status) {
+    if (cudaEventRecord(p->dw_done, p->in) == cudaSuccess)
+      (void)cudaStreamWaitEvent(p->out, p->dw_done, 0);
+    if (cudaEventRecord(p->end, p->out) == cudaSuccess) (void)cudaStreamWaitEvent(s, p->end, 0);
+    return status;
+  };
+  if (!ok(cudaMemsetAsync(ws_dev, 0, GNORM_WORKSPACE_ALIGN, s)) || !ok(cudaEventRecord(p->start, s)))
+    return GNORM_ERR_CUDA;  // nothing forked yet
+  if (!ok(cudaStreamWaitEvent(p->in, p->start, 0)) || !ok(cudaStreamWaitEvent(p->out, p->start, 0)))
+    return fail(GNORM_ERR_CUDA);
   if (!ok(cudaMemcpyAsync(w_dev, w, static_cast<size_t>(N) * 2, cudaMemcpyHostToDevice, p->in)))
-    return GNORM_ERR_CUDA;
+    return fail(GNORM_ERR_CUDA);
   const size_t row_b = static_cast<size_t>(N) * 2;
   for (int k = 0; k < L.chunks; ++k) {
     const int64_t r0 = k * L.rows_per_chunk;
@@ -217,32 +226,32 @@ extern "C" int gnorm_ckpt_step_host(const void* x, const void* g, const void* w,
         !ok(cudaMemcpyAsync(g_dev + o, static_cast<const uint8_t*>(g) + o, n, cudaMemcpyHostToDevice, p->in)) ||
         !ok(cudaMemcpyAsync(dy_dev + o, static_cast<const uint8_t*>(dy) + o, n, cudaMemcpyHostToDevice, p->in)) ||
         !ok(cudaEventRecord(p->in_done[k], p->in)))
-      return GNORM_ERR_CUDA;
+      return fail(GNORM_ERR_CUDA);
   }
   for (int k = 0; k < L.chunks; ++k) {
     const int64_t r0 = k * L.rows_per_chunk;
     const int64_t rows = (M - r0 < L.rows_per_chunk) ? M - r0 : L.rows_per_chunk;
     const size_t o = static_cast<size_t>(r0) * row_b, n = static_cast<size_t>(rows) * row_b;
-    if (!ok(cudaStreamWaitEvent(s, p->in_done[k], 0))) return GNORM_ERR_CUDA;
+    if (!ok(cudaStreamWaitEvent(s, p->in_done[k], 0))) return fail(GNORM_ERR_CUDA);
     st = gnorm_ckpt_step(x_dev + o, g_dev + o, w_dev, eps, dy_dev + o, y_dev + o, rstd_dev + r0,
                          dx_dev + o, dg_dev + o, dwc_dev + static_cast<size_t>(k) * N, 1,
                          deterministic, rows, N, ws_dev, L.ws_bytes, s);
-    if (st != GNORM_OK) return st;
+    if (st != GNORM_OK) return fail(st);
     if (!ok(cudaEventRecord(p->step_done[k], s)) || !ok(cudaStreamWaitEvent(p->out, p->step_done[k], 0)))
-      return GNORM_ERR_CUDA;
+      return fail(GNORM_ERR_CUDA);
     if (!ok(cudaMemcpyAsync(static_cast<uint8_t*>(y) + o, y_dev + o, n, cudaMemcpyDeviceToHost, p->out)) ||
         !ok(cudaMemcpyAsync(rstd + r0, rstd_dev + r0, static_cast<size_t>(rows) * 4,
                             cudaMemcpyDeviceToHost, p->out)) ||
         !ok(cudaMemcpyAsync(static_cast<uint8_t*>(dx) + o, dx_dev + o, n, cudaMemcpyDeviceToHost, p->out)) ||
         !ok(cudaMemcpyAsync(static_cast<uint8_t*>(dg) + o, dg_dev + o, n, cudaMemcpyDeviceToHost, p->out)))
-      return GNORM_ERR_CUDA;
+      return fail(GNORM_ERR_CUDA);
   }
   // dw: the chunks' FP32 rows summed in chunk order, then copied out; join.
   st = gnorm_dw_reduce(dwc_dev, L.chunks, N, dw_dev, dw_fp32, s);
-  if (st != GNORM_OK) return st;
+  if (st != GNORM_OK) return fail(st);
   if (!ok(cudaEventRecord(p->dw_done, s)) || !ok(cudaStreamWaitEvent(p->out, p->dw_done, 0)) ||
       !ok(cudaMemcpyAsync(dw, dw_dev, dwb, cudaMemcpyDeviceToHost, p->out)) ||
       !ok(cudaEventRecord(p->end, p->out)) || !ok(cudaStreamWaitEvent(s, p->end, 0)))
-    return GNORM_ERR_CUDA;
+    return fail(GNORM_ERR_CUDA);
   return GNORM_OK;
 }

@@ -227,7 +227,10 @@ GNORM_API int gnorm_ckpt_step(const void* x, const void* g, const void* w, float
  *   the call: it returns once everything is enqueued; the caller's stream waits for the
  *   last copy out, so synchronising the stream (or an event recorded on it afterwards)
  *   means every host output is written.  Errors: as gnorm_ckpt_step, and GNORM_ERR_WORKSPACE
- *   for a missing, misaligned or small dev_buf.  Not meant for CUDA graph capture.
+ *   for a missing, misaligned or small dev_buf.  A call that fails after it has started
+ *   enqueueing still joins its copy streams back into `stream` before it returns, so the
+ *   copies already queued are ordered on `stream` as well; its outputs are then undefined.
+ *   Not meant for CUDA graph capture.
  */
 GNORM_API int gnorm_ckpt_step_host(const void* x, const void* g, const void* w, float eps,
                                    const void* dy, void* y, float* rstd, void* dx, void* dg,
