@@ -12,8 +12,8 @@
 // Design: the same persistent, warp-specialised TMA pipeline as the forward, with three
 // tensors (dy, x, g) per stage (packed or strided rows).  Pass 1 recomputes xhat and the gate from shared memory,
 // writes dg, accumulates the row dot product sum(u xhat) and this thread's dw columns in
-// FP32 registers (arithmetic on packed FP32 pairs), and keeps u in registers; after the row
-// reduction pass 2 re-reads x and writes dx.  The producer warp also stages the rows' rstd
+// FP32 registers (arithmetic on packed FP32 pairs), and keeps u and xhat in registers; after
+// the row reduction pass 2 writes dx.  The producer warp also stages the rows' rstd
 // with 4-byte asynchronous copies tracked by the same stage barrier.  At the end each CTA adds its row groups' dw accumulators in a fixed order into one
 // FP32 partial row [P, N] in the workspace.  A second pass sums the P partials in a fixed
 // order and writes dw once, rounded to BF16 or kept in FP32: by default a second launch whose
@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
     gated_rmsnorm_bwd_kernel(const __grid_constant__ BwdArgs a) {
   constexpr int kNCT = consumer_threads_for(1, TPR, CPT);
   constexpr int kGroups = kNCT / TPR;
+  constexpr bool kKeepXhat = kNCT <= 256 || CPT == 1;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
@@ -371,6 +372,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
 
       // pass 1: recompute xhat and the gate; dg; row dot product; dw accumulators
       float2 u[CPT][4];
+      float2 xh[CPT][4];  // xhat, kept for pass 2 where the registers allow it
       float part[CPT];
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
@@ -378,7 +380,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
         if (cval[k]) {
           const int c = k * TPR + lr;
           const size_t off = roff + static_cast<size_t>(c) * 16;
-          float2 dyp[4], xp[4], gp[4], dgp[4], xh[4];
+          float2 dyp[4], xp[4], gp[4], dgp[4];
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sg + off), gp);
@@ -390,13 +392,13 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
             const float2 t = mul2(dyp[i], xhat);                    // dy xhat
             const float2 ue = mul2(mul2(dyp[i], wp[k][i]), silu);    // dy w s
             u[k][i] = ue;
-            xh[i] = xhat;
+            xh[k][i] = xhat;
             if (valid) dwacc[k][i] = fma2(t, silu, dwacc[k][i]);
             // sigmoid' = sigmoid (1 + g (1 - sigmoid))
             const float2 bracket = gate_grad_bracket(gp[i], sgm);
             dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), bracket);
           }
-          part[k] = chunk_dot(u[k], xh);  // this chunk's share of sum(u xhat)
+          part[k] = chunk_dot(u[k], xh[k]);  // this chunk's share of sum(u xhat)
           if (valid)
             *reinterpret_cast<uint4*>(a.dg + grow * a.lddg + c * 8) = pairs_to_bf16x8(dgp);
         }
@@ -405,18 +407,24 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
       slot ^= 1;
       const float2 nrc2 = splat2(-(r * (dot * a.inv_n)));
 
-      // pass 2: dx = r u - (r c) xhat, with xhat recomputed from the staged x (this keeps
-      // u, w and the dw accumulators as the only per-element registers)
+      // pass 2: dx = r u - (r c) xhat.  xhat comes from pass 1's registers, except for the
+      // widest rows (544 threads per CTA cap the registers), which recompute it from the
+      // staged x -- the same product, so the same bits.
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
         if (cval[k]) {
           const int c = k * TPR + lr;
-          float2 xp[4], dxp[4];
-          bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(c) * 16),
-                          xp);
+          float2 dxp[4];
+          if constexpr (kKeepXhat) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            dxp[i] = fma2(nrc2, mul2(xp[i], r2), mul2(r2, u[k][i]));
+            for (int i = 0; i < 4; ++i) dxp[i] = fma2(nrc2, xh[k][i], mul2(r2, u[k][i]));
+          } else {
+            float2 xp[4];
+            bf16x8_to_pairs(
+                *reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(c) * 16), xp);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) dxp[i] = fma2(nrc2, mul2(xp[i], r2), mul2(r2, u[k][i]));
+          }
           if (valid)
             *reinterpret_cast<uint4*>(a.dx + grow * a.lddx + c * 8) = pairs_to_bf16x8(dxp);
         }
