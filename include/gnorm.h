@@ -210,8 +210,8 @@ GNORM_API int gnorm_ckpt_step(const void* x, const void* g, const void* w, float
  * written to host memory; all rows packed.  The rows are processed in chunks (about 4 MiB of
  * x, g and dy each; 32 MiB when x, g and dy exceed 64 MiB) as a pipeline over the caller's
  * stream and two copy streams the library creates once per device: chunk k's inputs are
- * copied in while chunk k-1's step runs and
- * earlier chunks' outputs are copied out, so both directions of the host link work at once.
+ * copied in while chunk k-1's step runs and earlier chunks' outputs are copied out, so both
+ * directions of the host link work at once.
  * Each chunk runs gnorm_ckpt_step with an FP32 dw of its own rows; dw is the fixed-order sum
  * of those rows (gnorm_dw_reduce).  y, rstd, dx and dg are bitwise equal to gnorm_ckpt_step's;
  * dw is too when there is one chunk (M x N x 6 bytes <= 4 MiB), and otherwise is rounded
