@@ -64,6 +64,12 @@ def ckpt_bytes(M, N, dw_fp32):
     return 2 * fwd_bytes(M, N) + bwd_bytes(M, N, dw_fp32)
 
 
+def fwd_bwd_bytes(M, N, dw_fp32):
+    """The fused forward + backward of the same rows: read x, g, dy; write y, rstd, dx, dg
+    (12N + 4 per row), w once and dw."""
+    return M * (12 * N + 4) + 2 * N + N * (4 if dw_fp32 else 2)
+
+
 # ----------------------------------------------------------------------------- env
 
 def dist_env():
@@ -391,7 +397,9 @@ class Problem:
     """Device tensors of one workload and CUDA graphs of its three operations (fwdg, bwdg,
     ckptg, as the pages name them)."""
 
-    def __init__(self, torch, gn, dev, stream, wl, det, fp32, seed_offset=0, graphs=True):
+    def __init__(self, torch, gn, dev, stream, wl, det, fp32, seed_offset=0, graphs=True,
+                 knobs=None):
+        knobs = knobs or {}
         self.torch, self.gn, self.wl = torch, gn, wl
         self.M, self.N, self.eps = wl.M, wl.N, wl.eps
         self.det, self.fp32 = det, fp32
@@ -411,10 +419,15 @@ class Problem:
         self.plan_f = gn.gnorm_plan_query(0, wl.M, wl.N, det, sms)
         self.plan_b = gn.gnorm_plan_query(1, wl.M, wl.N, det, sms)
         self.bwd_launches = 1 + (0 if self.plan_b["fused_reduce"] else 1)
-        self.launches = {"ckpt": 2 + self.bwd_launches, "bwd": self.bwd_launches, "fwd": 1}
+        # the recompute forward and the backward run as one kernel where the backward's
+        # plan stages its rows (and the fuse_fwd_bwd knob does not say otherwise)
+        self.fused = (not self.plan_b["direct_loads"]) and knobs.get("fuse_fwd_bwd", 0) != 2
+        fb = self.bwd_launches + (0 if self.fused else 1)
+        self.launches = {"ckpt": 1 + fb, "fwd_bwd": fb, "bwd": self.bwd_launches, "fwd": 1}
         self.graphs = {name: capture_graph(torch, dev, stream, fn)
-                       for name, fn in (("ckpt", self.op_ckpt), ("bwd", self.op_bwd),
-                                        ("fwd", self.op_fwd))} if graphs else {}
+                       for name, fn in (("ckpt", self.op_ckpt), ("fwd_bwd", self.op_fwd_bwd),
+                                        ("bwd", self.op_bwd), ("fwd", self.op_fwd))
+                       } if graphs else {}
 
     def op_fwd(self):
         self.gn.gnorm_fwd(self.x, self.g, self.w, self.eps, y=self.y, rstd=self.rstd)
@@ -423,6 +436,11 @@ class Problem:
         self.gn.gnorm_bwd(self.dy, self.x, self.g, self.w, self.rstd, dx=self.dx, dg=self.dg,
                           dw=self.dw, dw_fp32=self.fp32, deterministic=self.det,
                           workspace_buf=self.ws)
+
+    def op_fwd_bwd(self):
+        self.gn.gnorm_fwd_bwd(self.x, self.g, self.w, self.eps, self.dy, y=self.y,
+                              rstd=self.rstd, dx=self.dx, dg=self.dg, dw=self.dw,
+                              dw_fp32=self.fp32, deterministic=self.det, workspace_buf=self.ws)
 
     def op_ckpt(self):
         self.gn.gnorm_ckpt_step(self.x, self.g, self.w, self.eps, self.dy, y=self.y,
@@ -435,16 +453,24 @@ class Problem:
 
     def bytes(self):
         return {"fwd": fwd_bytes(self.M, self.N), "bwd": bwd_bytes(self.M, self.N, self.fp32),
+                "fwd_bwd": fwd_bwd_bytes(self.M, self.N, self.fp32),
                 "ckpt": ckpt_bytes(self.M, self.N, self.fp32)}
+
+    def step_dram_bytes(self):
+        """Bytes the checkpointed step must move as this library runs it: the forward, then
+        the fused forward + backward (or the forward and the backward apart)."""
+        b = self.bytes()
+        return b["fwd"] + (b["fwd_bwd"] if self.fused else b["fwd"] + b["bwd"])
 
     def release(self):
         self.graphs.clear()
 
 
 def op_times(timer, prob, reps):
-    """Mean device microseconds per replay of fwdg, bwdg and ckptg."""
+    """Mean device microseconds per replay of fwdg, bwdg, the fused forward + backward and
+    ckptg."""
     out = {}
-    for name in ("fwd", "bwd", "ckpt"):
+    for name in ("fwd", "bwd", "fwd_bwd", "ckpt"):
         timer.run(prob.graphs[name], 3)
         total, _ = timer.run(prob.graphs[name], reps)
         out[name] = total / reps * 1e3
@@ -471,7 +497,7 @@ def run_ours(args, wl):
     stream = torch.cuda.current_stream(dev)
     l2 = l2_bytes(torch, dev)
     flush = torch.empty(max(L2_FLUSH_BYTES, 2 * l2), dtype=torch.uint8, device=dev)
-    prob = Problem(torch, gn, dev, stream, wl, det, fp32, seed_offset=rank)
+    prob = Problem(torch, gn, dev, stream, wl, det, fp32, seed_offset=rank, knobs=knobs)
     M, N = prob.M, prob.N
     # The smallest operation's inputs: the forward reads x and g.
     streamed = (not args.flush) and 2 * M * N * 2 > l2
@@ -507,13 +533,14 @@ def run_ours(args, wl):
     # (this also counts each replay's own launch latency)
     cold_reps = max(10, min(K, 100))
     us_cold = {name: prob_t * 1e3 for name, prob_t in
-               ((n, timer.cold(prob.graphs[n], cold_reps)) for n in ("fwd", "bwd", "ckpt"))}
+               ((n, timer.cold(prob.graphs[n], cold_reps))
+                for n in ("fwd", "bwd", "fwd_bwd", "ckpt"))}
     per_config = {}
     if args.per_config and world == 1:
         for name in PER_CONFIG_WORKLOADS:
             if name == wl.name:
                 continue
-            other = Problem(torch, gn, dev, stream, WORKLOADS[name], det, fp32)
+            other = Problem(torch, gn, dev, stream, WORKLOADS[name], det, fp32, knobs=knobs)
             o_streamed = (not args.flush) and 2 * other.M * other.N * 2 > l2
             o_timer = Timer(torch, stream, flush, o_streamed)
             t = op_times(o_timer, other, args.per_config_steps)
@@ -521,7 +548,9 @@ def run_ours(args, wl):
             per_config[name] = {
                 "M": other.M, "N": other.N, "us": t,
                 "gbs": {k: b[k] / (t[k] * 1e-6) / 1e9 for k in t},
-                "frac_of_peak": {k: b[k] / (t[k] * 1e-6) / 1e9 / peak for k in t},
+                "frac_of_peak": {k: b[k] / (t[k] * 1e-6) / 1e9 / peak for k in t if k != "ckpt"},
+                "frac_of_peak_ckpt_dram": other.step_dram_bytes() / (t["ckpt"] * 1e-6) / 1e9
+                                          / peak,
                 "fwd_kernel": other.fwd_kernel(),
                 "l2": "inputs larger than L2, replays back to back" if o_streamed
                       else "L2 flushed before every replay",
@@ -579,12 +608,33 @@ def run_ours(args, wl):
     b = prob.bytes()
     gbs = {k: b[k] / (us[k] * 1e-6) / 1e9 for k in us}
     gbs_cold = {k: b[k] / (us_cold[k] * 1e-6) / 1e9 for k in us_cold}
-    fwd_traffic = profiled_traffic("fwd_kernel", wl.name)
-    bwd_traffic = profiled_traffic("bwd_kernel", wl.name)
-    # device time of one step by operation, from the standalone replays: the forward
-    # kernel (twice) and the backward operation (kernel + second pass)
-    step_us = 2 * us["fwd"] + us["bwd"]
-    shares = {"fwd_kernel_x2": 2 * us["fwd"] / step_us, "bwd_op": us["bwd"] / step_us}
+    traffic = {k: profiled_traffic(f"{k}_kernel", wl.name) for k in ("fwd", "bwd", "fwd_bwd")}
+    # device time of one step by operation, from the standalone replays: the forward kernel,
+    # then the fused forward + backward (kernel + dw pass), or, unfused, the forward twice
+    # and the backward (kernel + dw pass)
+    if prob.fused:
+        step_us = us["fwd"] + us["fwd_bwd"]
+        shares = {"fwd_kernel": us["fwd"] / step_us, "fwd_bwd_op": us["fwd_bwd"] / step_us}
+    else:
+        step_us = 2 * us["fwd"] + us["bwd"]
+        shares = {"fwd_kernel_x2": 2 * us["fwd"] / step_us, "bwd_op": us["bwd"] / step_us}
+    fwd_name = f"{prob.fwd_kernel()} (one launch per fwdg replay)"
+    objs = {
+        "fwd": fwd_name,
+        "bwd": "gnorm_bwd (backward kernel + dw second pass, one bwdg replay)",
+        "fwd_bwd": ("gnorm_fwd_bwd (the forward fused into the backward kernel, + dw second "
+                    "pass; one replay)" if prob.fused else
+                    "gnorm_fwd_bwd (forward kernel, backward kernel, dw pass; one replay)"),
+    }
+
+    def roofline_of(key):
+        return {"bound": "hbm", "kernel": objs[key], "achieved": gbs[key], "peak": peak,
+                "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs[key] / peak,
+                "algorithmic_bytes_per_launch": b[key], "traffic": traffic[key]}
+
+    # the operation with the largest share of the step's device time
+    dominant = "fwd_bwd" if (prob.fused and us["fwd_bwd"] > us["fwd"]) else "fwd"
+    dram_step = prob.step_dram_bytes()
     cpu = cpu_all = None
     if not args.no_cpu_baseline and world == 1:  # the CPU baseline runs at N = 1 only
         c_gbs, c_rows, c_reps, c_sec = time_oracle(wl, args.cpu_seconds)
@@ -607,8 +657,9 @@ def run_ours(args, wl):
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "M": M, "N": N, "eps": prob.eps,
-                   "step": "checkpointed step as one CUDA graph: fwd, fwd (recompute), "
-                           "bwd + dw reduction",
+                   "step": "checkpointed step as one CUDA graph: fwd, then the recompute "
+                           "fwd and the bwd (fused into one kernel where the backward stages "
+                           "its rows), + dw reduction",
                    "deterministic": det, "dw": "fp32" if fp32 else "bf16",
                    "l2": l2_note,
                    "parallelism": f"dp{world} (independent rows per rank, no collective)",
@@ -620,25 +671,29 @@ def run_ours(args, wl):
                    "each of ckptg, fwdg, bwdg replayed from its own CUDA graph between two "
                    "CUDA events after an L2 flush"),
         "gbs": gbs,
-        "frac_of_peak": {k: v / peak for k, v in gbs.items()},
+        # each operation's algorithmic bytes over its time, against the HBM peak; for the
+        # step the bytes are the counted 2 x forward + backward (see step_bytes_note), so its
+        # fraction of the HBM peak is the DRAM one below
+        "frac_of_peak": {k: v / peak for k, v in gbs.items() if k != "ckpt"},
+        "frac_of_peak_ckpt_dram": (dram_step / (us["ckpt"] * 1e-6) / 1e9) / peak,
         "us_per_call_cold_l2": us_cold,
-        "frac_of_peak_cold_l2": {k: v / peak for k, v in gbs_cold.items()},
+        "frac_of_peak_cold_l2": {k: v / peak for k, v in gbs_cold.items() if k != "ckpt"},
         "cold_l2_note": (f"{cold_reps} replays each after a {flush.numel() >> 20} MiB L2 flush, "
                          "events around each replay, so each also counts its graph's launch "
                          "latency"),
-        "roofline": {"bound": "hbm",
-                     "kernel": f"{prob.fwd_kernel()} (one launch per fwdg replay)",
-                     "achieved": gbs["fwd"], "peak": peak, "peak_kind": peak_kind,
-                     "unit": "GB/s", "frac": gbs["fwd"] / peak,
-                     "algorithmic_bytes_per_launch": b["fwd"],
-                     "traffic": fwd_traffic},
-        "roofline_bwd": {"bound": "hbm",
-                         "kernel": "gnorm_bwd (backward kernel + dw second pass, one bwdg "
-                                   "replay)",
-                         "achieved": gbs["bwd"], "peak": peak, "peak_kind": peak_kind,
-                         "unit": "GB/s", "frac": gbs["bwd"] / peak,
-                         "algorithmic_bytes_per_launch": b["bwd"],
-                         "traffic": bwd_traffic},
+        "roofline": roofline_of(dominant),
+        "roofline_fwd": roofline_of("fwd"),
+        "roofline_bwd": roofline_of("bwd"),
+        "roofline_fwd_bwd": roofline_of("fwd_bwd"),
+        "dram_bytes_per_step": dram_step,
+        "dram_gbs": dram_step * K * world / (total_ms * 1e-3) / 1e9,
+        "step_bytes_note": ("value counts the step as 2 x forward + backward (the pages' "
+                            "ckptg); the recompute forward runs inside the backward kernel, "
+                            "which reads x and g once for both, so the step moves "
+                            "dram_bytes_per_step to DRAM; dram_gbs is that over the same time"
+                            if prob.fused else
+                            "the step runs as three kernels: dram_bytes_per_step equals the "
+                            "counted bytes"),
         "step_shares": shares,
         "per_config": per_config or None,
         "cpu_baseline": cpu,
@@ -677,8 +732,9 @@ def run_profile(args, wl):
     if knobs:
         gn.gnorm_set_tuning(**knobs)
     prob = Problem(torch, gn, dev, torch.cuda.current_stream(dev), wl,
-                   not args.nondeterministic, not args.dw_bf16, graphs=False)
-    fn = {"fwd": prob.op_fwd, "bwd": prob.op_bwd, "ckpt": prob.op_ckpt}[args.profile_op]
+                   not args.nondeterministic, not args.dw_bf16, graphs=False, knobs=knobs)
+    fn = {"fwd": prob.op_fwd, "bwd": prob.op_bwd, "fwd_bwd": prob.op_fwd_bwd,
+          "ckpt": prob.op_ckpt}[args.profile_op]
     torch.cuda.synchronize()
     for _ in range(args.reps):
         fn()
@@ -716,7 +772,7 @@ def main(argv=None):
                     help="target duration of the reference (oracle) arm")
     ap.add_argument("--tune", action="append", default=[], metavar="KNOB=VALUE",
                     help="a gnorm_tuning knob for this run (repeatable; recorded in config)")
-    ap.add_argument("--profile-op", choices=("fwd", "bwd", "ckpt"),
+    ap.add_argument("--profile-op", choices=("fwd", "bwd", "fwd_bwd", "ckpt"),
                     help="run only this operation --reps times and exit (for ncu captures)")
     ap.add_argument("--reps", type=int, default=3)
     ap.add_argument("--rows", type=int, default=0,

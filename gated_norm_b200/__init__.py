@@ -18,6 +18,7 @@ from .gnorm import (  # noqa: F401
     gnorm_device_error,
     gnorm_dw_reduce,
     gnorm_fwd,
+    gnorm_fwd_bwd,
     gnorm_plan_query,
     gnorm_selftest_wait_timeout,
     gnorm_set_tuning,

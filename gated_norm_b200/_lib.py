@@ -54,7 +54,7 @@ class GnormTuning(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int) for name in (
         "stage_bytes", "max_stages", "ctas_per_sm", "disable_pdl", "threads_per_row",
         "chunks_per_thread", "l2_prefetch", "tail_reduce", "chain_prefetch",
-        "host_chunk_bytes", "fwd_direct", "bwd_direct")]
+        "host_chunk_bytes", "fwd_direct", "bwd_direct", "fuse_fwd_bwd")]
 
 
 class GnormFwdDesc(ctypes.Structure):
@@ -107,6 +107,9 @@ SIGNATURES = {
     "gnorm_ckpt_step_ex": (_int, [ctypes.POINTER(GnormFwdDesc), ctypes.POINTER(GnormBwdDesc), _vp]),
     "gnorm_ckpt_step": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
                                _i64, _vp, _sz, _vp]),
+    "gnorm_fwd_bwd_ex": (_int, [ctypes.POINTER(GnormFwdDesc), ctypes.POINTER(GnormBwdDesc), _vp]),
+    "gnorm_fwd_bwd": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int, _int, _i64,
+                             _i64, _vp, _sz, _vp]),
     "gnorm_ckpt_step_host": (_int, [_vp, _vp, _vp, _f32, _vp, _vp, _vp, _vp, _vp, _vp, _int,
                                     _int, _i64, _i64, _vp, _sz, _vp]),
     "gnorm_ckpt_step_host_bytes": (_sz, [_i64, _i64, _int]),

@@ -225,11 +225,15 @@ int enqueue_fwd(const DeviceInfo& d, const gnorm_fwd_desc& f, cudaStream_t strea
   return GNORM_OK;
 }
 
+// `fused`: the forward of the same rows runs in the same kernel (gnorm_fwd_bwd); it writes
+// fused->y and fused->rstd and reads no rstd.  Staged plans only (GNORM_ERR_UNSUPPORTED for a
+// direct-load plan, which the caller then runs as two kernels).
 int enqueue_bwd(const DeviceInfo& d, const gnorm_bwd_desc& b, cudaStream_t stream,
-                bool prefetch = false) {
+                bool prefetch = false, const gnorm_fwd_desc* fused = nullptr) {
   gnorm_plan plan;
   int st = make_plan(1, b.M, b.N, b.deterministic, d.num_sms, d.smem_optin, &plan);
   if (st != GNORM_OK) return st;
+  if (fused != nullptr && plan.direct_loads) return GNORM_ERR_UNSUPPORTED;
   uint8_t* wsb = static_cast<uint8_t*>(b.workspace);
   BwdArgs a;
   a.dy = static_cast<const uint16_t*>(b.dy);
@@ -261,6 +265,13 @@ int enqueue_bwd(const DeviceInfo& d, const gnorm_bwd_desc& b, cudaStream_t strea
   a.prefetch = prefetch ? 1 : 0;
   a.l2_prefetch = plan.l2_prefetch;
   a.err = d.err_word;
+  if (fused != nullptr) {
+    a.fused_fwd = 1;
+    a.y = static_cast<uint16_t*>(fused->y);
+    a.ldy = fused->ldy;
+    a.rstd_out = fused->rstd;
+    a.eps = fused->eps;
+  }
   const int R = plan.rows_per_stage;
   if (!plan.direct_loads) {
     if (rows_map(&a.map_dy, b.dy, b.M, b.N, b.lddy, R)) a.map_bits |= 1;
@@ -331,6 +342,77 @@ int check_workspace(const DeviceInfo& d, int64_t M, int64_t N, int deterministic
   return GNORM_OK;
 }
 
+// Validates a forward/backward descriptor pair of one set of rows (gnorm_ckpt_step_ex,
+// gnorm_fwd_bwd_ex): the backward's x, g, w, rstd must be NULL or the forward's, M and N
+// equal.  Resolves strides, fills *f and *b, checks aliasing and the workspace.  *noop is set
+// when M == 0 (dw has then been zeroed on `stream`).
+int check_fwd_bwd(const gnorm_fwd_desc* fwd, const gnorm_bwd_desc* bwd, void* stream,
+                  gnorm_fwd_desc* f_out, gnorm_bwd_desc* b_out, DeviceInfo* d, bool* noop) {
+  *noop = false;
+  if (fwd == nullptr || bwd == nullptr) return GNORM_ERR_NULL;
+  gnorm_fwd_desc f = *fwd;
+  gnorm_bwd_desc b = *bwd;
+  if (b.M != f.M || b.N != f.N) return GNORM_ERR_ARG;
+  // The backward reads the forward's x, g, w and the rstd it writes.
+  if ((b.x && (b.x != f.x || (b.ldx ? b.ldx : f.N) != (f.ldx ? f.ldx : f.N))) ||
+      (b.g && (b.g != f.g || (b.ldg ? b.ldg : f.N) != (f.ldg ? f.ldg : f.N))) ||
+      (b.w && (b.w != f.w || b.w_fp32 != f.w_fp32)) || (b.rstd && b.rstd != f.rstd))
+    return GNORM_ERR_ARG;
+  b.x = f.x;
+  b.ldx = f.ldx;
+  b.g = f.g;
+  b.ldg = f.ldg;
+  b.w = f.w;
+  b.w_fp32 = f.w_fp32;
+  b.rstd = f.rstd;
+  bool noop_f = false, noop_b = false;
+  int st = check_fwd(&f, &noop_f);
+  if (st != GNORM_OK) return st;
+  st = check_bwd(&b, &noop_b);
+  if (st != GNORM_OK) return st;
+  const size_t dw_bytes = static_cast<size_t>(b.N) * (b.dw_fp32 ? 4 : 2);
+  if (noop_b) {
+    *noop = true;
+    return cudaMemsetAsync(b.dw, 0, dw_bytes, as_stream(stream)) == cudaSuccess ? GNORM_OK
+                                                                                 : GNORM_ERR_CUDA;
+  }
+  const Region in[] = {mat(f.x, f.M, f.N, f.ldx), mat(f.g, f.M, f.N, f.ldg),
+                       span(f.w, w_bytes(f.N, f.w_fp32)), mat(b.dy, b.M, b.N, b.lddy)};
+  const Region out[] = {mat(f.y, f.M, f.N, f.ldy),
+                        span(f.rstd, static_cast<size_t>(f.M) * 4),
+                        mat(b.dx, b.M, b.N, b.lddx),
+                        mat(b.dg, b.M, b.N, b.lddg),
+                        span(b.dw, dw_bytes),
+                        span(b.workspace, b.workspace_bytes)};
+  if (any_alias(in, 4, out, 6)) return GNORM_ERR_ALIAS;
+  st = device_info(d);
+  if (st != GNORM_OK) return st;
+  st = check_workspace(*d, b.M, b.N, b.deterministic, b.workspace, b.workspace_bytes);
+  if (st != GNORM_OK) return st;
+  *f_out = f;
+  *b_out = b;
+  return GNORM_OK;
+}
+
+// The forward of a set of rows followed by its backward.  One fused kernel (the staged
+// backward plan) or, for direct-load plans or when the fuse_fwd_bwd knob says so, the forward
+// kernel then the backward kernel.  `chain`: the previous kernel on the stream writes none of
+// x, g, dy (the first forward of a checkpointed step), so input copies may start early.
+int enqueue_fwd_bwd(const DeviceInfo& d, const gnorm_fwd_desc& f, const gnorm_bwd_desc& b,
+                    cudaStream_t s, bool chain) {
+  const int fk = get_tuning().fuse_fwd_bwd;
+  const bool fuse = fk == 1 ? true : (fk == 2 ? false : kDefaultFuseFwdBwd != 0);
+  if (fuse) {
+    const int st = enqueue_bwd(d, b, s, chain, &f);
+    if (st != GNORM_ERR_UNSUPPORTED) return st;
+  }
+  // Two kernels: the forward, then the backward, which only reads rstd once the forward
+  // has ended (neither writes x, g or dy, so the backward's input copies may start early).
+  int st = enqueue_fwd(d, f, s, chain);
+  if (st != GNORM_OK) return st;
+  return enqueue_bwd(d, b, s, chain);
+}
+
 }  // namespace
 }  // namespace gnorm
 
@@ -379,56 +461,31 @@ int gnorm_bwd_ex(const gnorm_bwd_desc* desc, void* stream) {
 }
 
 int gnorm_ckpt_step_ex(const gnorm_fwd_desc* fwd, const gnorm_bwd_desc* bwd, void* stream) {
-  if (fwd == nullptr || bwd == nullptr) return GNORM_ERR_NULL;
-  gnorm_fwd_desc f = *fwd;
-  gnorm_bwd_desc b = *bwd;
-  if (b.M != f.M || b.N != f.N) return GNORM_ERR_ARG;
-  // The backward reads the forward's x, g, w and the rstd it writes.
-  if ((b.x && (b.x != f.x || (b.ldx ? b.ldx : f.N) != (f.ldx ? f.ldx : f.N))) ||
-      (b.g && (b.g != f.g || (b.ldg ? b.ldg : f.N) != (f.ldg ? f.ldg : f.N))) ||
-      (b.w && (b.w != f.w || b.w_fp32 != f.w_fp32)) || (b.rstd && b.rstd != f.rstd))
-    return GNORM_ERR_ARG;
-  b.x = f.x;
-  b.ldx = f.ldx;
-  b.g = f.g;
-  b.ldg = f.ldg;
-  b.w = f.w;
-  b.w_fp32 = f.w_fp32;
-  b.rstd = f.rstd;
-  bool noop_f = false, noop_b = false;
-  int st = check_fwd(&f, &noop_f);
-  if (st != GNORM_OK) return st;
-  st = check_bwd(&b, &noop_b);
-  if (st != GNORM_OK) return st;
-  const size_t dw_bytes = static_cast<size_t>(b.N) * (b.dw_fp32 ? 4 : 2);
-  if (noop_b)
-    return cudaMemsetAsync(b.dw, 0, dw_bytes, as_stream(stream)) == cudaSuccess ? GNORM_OK
-                                                                                 : GNORM_ERR_CUDA;
-  const Region in[] = {mat(f.x, f.M, f.N, f.ldx), mat(f.g, f.M, f.N, f.ldg),
-                       span(f.w, w_bytes(f.N, f.w_fp32)), mat(b.dy, b.M, b.N, b.lddy)};
-  const Region out[] = {mat(f.y, f.M, f.N, f.ldy),
-                        span(f.rstd, static_cast<size_t>(f.M) * 4),
-                        mat(b.dx, b.M, b.N, b.lddx),
-                        mat(b.dg, b.M, b.N, b.lddg),
-                        span(b.dw, dw_bytes),
-                        span(b.workspace, b.workspace_bytes)};
-  if (any_alias(in, 4, out, 6)) return GNORM_ERR_ALIAS;
+  gnorm_fwd_desc f;
+  gnorm_bwd_desc b;
   DeviceInfo d;
-  st = device_info(&d);
-  if (st != GNORM_OK) return st;
-  st = check_workspace(d, b.M, b.N, b.deterministic, b.workspace, b.workspace_bytes);
-  if (st != GNORM_OK) return st;
+  bool noop = false;
+  int st = check_fwd_bwd(fwd, bwd, stream, &f, &b, &d, &noop);
+  if (st != GNORM_OK || noop) return st;
   const cudaStream_t s = as_stream(stream);
-  // The second forward (the recompute) follows the first, which writes only y and rstd;
-  // the backward follows it and reads rstd only after it ends.  Neither predecessor writes
-  // x, g or dy (outputs may not overlap inputs), so those copies may start early.
+  // The first forward, then the recompute forward fused with the backward (or the two as
+  // separate kernels).  The first forward writes only y and rstd; the second forward and
+  // the backward read x, g and dy, which it cannot overlap, so their copies may start early.
   const int cp = get_tuning().chain_prefetch;
   const bool chain = cp == 1 ? true : (cp == 2 ? false : kDefaultChainPrefetch != 0);
   st = enqueue_fwd(d, f, s);
   if (st != GNORM_OK) return st;
-  st = enqueue_fwd(d, f, s, chain);
-  if (st != GNORM_OK) return st;
-  return enqueue_bwd(d, b, s, chain);
+  return enqueue_fwd_bwd(d, f, b, s, chain);
+}
+
+int gnorm_fwd_bwd_ex(const gnorm_fwd_desc* fwd, const gnorm_bwd_desc* bwd, void* stream) {
+  gnorm_fwd_desc f;
+  gnorm_bwd_desc b;
+  DeviceInfo d;
+  bool noop = false;
+  int st = check_fwd_bwd(fwd, bwd, stream, &f, &b, &d, &noop);
+  if (st != GNORM_OK || noop) return st;
+  return enqueue_fwd_bwd(d, f, b, as_stream(stream), false);
 }
 
 int gnorm_fwd(const void* x, const void* g, const void* w, float eps, void* y, float* rstd,
@@ -502,6 +559,27 @@ int gnorm_ckpt_step(const void* x, const void* g, const void* w, float eps, cons
   const gnorm_bwd_desc b = packed_bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic,
                                            M, N, workspace, workspace_bytes);
   return gnorm_ckpt_step_ex(&f, &b, stream);
+}
+
+int gnorm_fwd_bwd(const void* x, const void* g, const void* w, float eps, const void* dy,
+                  void* y, float* rstd, void* dx, void* dg, void* dw, int dw_fp32,
+                  int deterministic, int64_t M, int64_t N, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  gnorm_fwd_desc f = {};
+  f.x = x;
+  f.ldx = N;
+  f.g = g;
+  f.ldg = N;
+  f.w = w;
+  f.eps = eps;
+  f.y = y;
+  f.ldy = N;
+  f.rstd = rstd;
+  f.M = M;
+  f.N = N;
+  const gnorm_bwd_desc b = packed_bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic,
+                                           M, N, workspace, workspace_bytes);
+  return gnorm_fwd_bwd_ex(&f, &b, stream);
 }
 
 int gnorm_dw_reduce(const float* partials, int64_t P, int64_t N, void* dw, int dw_fp32,
@@ -592,6 +670,7 @@ void gnorm_set_tuning(const gnorm_tuning* tuning) {
     k.host_chunk_bytes = clamp0(k.host_chunk_bytes);
     k.fwd_direct = tri(k.fwd_direct);
     k.bwd_direct = tri(k.bwd_direct);
+    k.fuse_fwd_bwd = tri(k.fuse_fwd_bwd);
   }
   set_tuning(k);
 }

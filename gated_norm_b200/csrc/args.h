@@ -59,6 +59,13 @@ struct BwdArgs {
   int prefetch = 0;  // 1: the first stages' dy, x, g may be copied before the previous grid ends
   int l2_prefetch = 0;  // 1: also warm L2 with the block the CTA loads after the ring's
   unsigned* err;
+  // Fused forward (gnorm_fwd_bwd): the kernel computes each row's rstd itself from the
+  // staged x, writes it to rstd_out and y = x r w silu(g) to y, and reads no rstd.
+  int fused_fwd = 0;
+  uint16_t* y = nullptr;
+  long long ldy = 0;
+  float* rstd_out = nullptr;
+  float eps = 0.f;
 };
 
 }  // namespace gnorm

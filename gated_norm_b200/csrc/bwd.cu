@@ -5,21 +5,25 @@
 
 namespace gnorm {
 
-template <int TPR, int CPT, bool kWFp32>
-static cudaError_t launch_bwd_weight(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream,
+template <int TPR, int CPT, bool kWFp32, bool kFusedFwd>
+static cudaError_t launch_bwd_variant(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream,
                                       bool pdl) {
-  const void* k = reinterpret_cast<const void*>(&gated_rmsnorm_bwd_kernel<TPR, CPT, kWFp32>);
+  const void* k =
+      reinterpret_cast<const void*>(&gated_rmsnorm_bwd_kernel<TPR, CPT, kWFp32, kFusedFwd>);
   cudaError_t e = ensure_smem_limit(k, p.smem_bytes);
   if (e != cudaSuccess) return e;
-  return launch_kernel(gated_rmsnorm_bwd_kernel<TPR, CPT, kWFp32>, p.grid,
+  return launch_kernel(gated_rmsnorm_bwd_kernel<TPR, CPT, kWFp32, kFusedFwd>, p.grid,
                        consumer_threads_for(1, TPR, CPT) + 32, p.smem_bytes, stream, pdl, a);
 }
 
 template <int TPR, int CPT>
 static cudaError_t launch_bwd_geometry(const gnorm_plan& p, const BwdArgs& a,
                                        cudaStream_t stream, bool pdl) {
-  return a.w_fp32 ? launch_bwd_weight<TPR, CPT, true>(p, a, stream, pdl)
-                  : launch_bwd_weight<TPR, CPT, false>(p, a, stream, pdl);
+  if (a.fused_fwd)
+    return a.w_fp32 ? launch_bwd_variant<TPR, CPT, true, true>(p, a, stream, pdl)
+                    : launch_bwd_variant<TPR, CPT, false, true>(p, a, stream, pdl);
+  return a.w_fp32 ? launch_bwd_variant<TPR, CPT, true, false>(p, a, stream, pdl)
+                  : launch_bwd_variant<TPR, CPT, false, false>(p, a, stream, pdl);
 }
 
 template <int TPR>
@@ -34,6 +38,7 @@ static cudaError_t launch_bwd_direct(const gnorm_plan& p, const BwdArgs& a, cuda
 
 cudaError_t launch_bwd(const gnorm_plan& p, const BwdArgs& a, cudaStream_t stream, bool pdl) {
   if (p.direct_loads) {
+    if (a.fused_fwd) return cudaErrorInvalidConfiguration;  // staged kernels only
     if (p.chunks_per_thread != 1) return cudaErrorInvalidConfiguration;
     switch (p.threads_per_row) {
       case 4: return launch_bwd_direct<4>(p, a, stream, pdl);

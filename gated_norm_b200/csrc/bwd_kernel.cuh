@@ -183,7 +183,10 @@ __global__ void __launch_bounds__(kReduceThreads)
   if (work_counter != nullptr && blockIdx.x == 0 && threadIdx.x == 0) *work_counter = 0ull;
 }
 
-template <int TPR, int CPT, bool kWFp32>
+// kFusedFwd: the forward of the same rows in the same pass (gnorm_fwd_bwd) -- each row's
+// rstd is computed from the staged x (the forward's arithmetic and order, so the same bits),
+// written out with y, and used for the backward; no rstd is read.
+template <int TPR, int CPT, bool kWFp32, bool kFusedFwd>
 __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ctas_per_sm(1, TPR, CPT))
     gated_rmsnorm_bwd_kernel(const __grid_constant__ BwdArgs a) {
   constexpr int kNCT = consumer_threads_for(1, TPR, CPT);
@@ -309,8 +312,10 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
           }
         }
       }
-      float* srs = reinterpret_cast<float*>(st + 3u * tensor_bytes);
-      for (int i = lane; i < rows; i += 32) async_copy_4(srs + i, a.rstd + r0 + i);
+      if constexpr (!kFusedFwd) {
+        float* srs = reinterpret_cast<float*>(st + 3u * tensor_bytes);
+        for (int i = lane; i < rows; i += 32) async_copy_4(srs + i, a.rstd + r0 + i);
+      }
       async_copies_arrive(&full[s]);
       if (lane == 0) mbar_arrive(&full[s]);
       if (++s == S) {
@@ -367,7 +372,28 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
       const int srow = valid ? row : 0;
       const size_t roff = static_cast<size_t>(srow) * N * 2;
       const long long grow = r0 + row;
-      const float r = srs[srow];
+      float r;
+      if constexpr (kFusedFwd) {
+        // the forward's row sum: sum of squares of the staged x, one partial per chunk
+        float sq[CPT];
+#pragma unroll
+        for (int k = 0; k < CPT; ++k) {
+          sq[k] = 0.f;
+          if (cval[k]) {
+            float2 xp[4];
+            bf16x8_to_pairs(
+                *reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(k * TPR + lr) * 16),
+                xp);
+            sq[k] = chunk_dot(xp, xp);
+          }
+        }
+        const float ss = row_sum<TPR>(combine_chunks<CPT>(sq), red_slots, group, lr, slot);
+        slot ^= 1;
+        r = rsqrtf(fmaf(ss, a.inv_n, a.eps));
+        if (valid && lr == 0) a.rstd_out[grow] = r;
+      } else {
+        r = srs[srow];
+      }
       const float2 r2 = splat2(r);
 
       // pass 1: recompute xhat and the gate; dg; row dot product; dw accumulators
@@ -380,7 +406,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
         if (cval[k]) {
           const int c = k * TPR + lr;
           const size_t off = roff + static_cast<size_t>(c) * 16;
-          float2 dyp[4], xp[4], gp[4], dgp[4];
+          float2 dyp[4], xp[4], gp[4], dgp[4], yp[4];
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sg + off), gp);
@@ -389,6 +415,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
             const float2 xhat = mul2(xp[i], r2);
             const float2 sgm = sigmoid2(gp[i]);
             const float2 silu = mul2(gp[i], sgm);
+            if constexpr (kFusedFwd) yp[i] = mul2(mul2(xhat, wp[k][i]), silu);  // the forward's y
             const float2 t = mul2(dyp[i], xhat);                    // dy xhat
             const float2 ue = mul2(mul2(dyp[i], wp[k][i]), silu);    // dy w s
             u[k][i] = ue;
@@ -399,8 +426,11 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
             dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), bracket);
           }
           part[k] = chunk_dot(u[k], xh[k]);  // this chunk's share of sum(u xhat)
-          if (valid)
+          if (valid) {
             *reinterpret_cast<uint4*>(a.dg + grow * a.lddg + c * 8) = pairs_to_bf16x8(dgp);
+            if constexpr (kFusedFwd)
+              *reinterpret_cast<uint4*>(a.y + grow * a.ldy + c * 8) = pairs_to_bf16x8(yp);
+          }
         }
       }
       const float dot = row_sum<TPR>(combine_chunks<CPT>(part), red_slots, group, lr, slot);

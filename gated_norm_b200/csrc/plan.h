@@ -41,6 +41,9 @@ constexpr int kBwdMaxStages = 3;
 constexpr int kDefaultL2Prefetch = 0;
 constexpr int kDefaultTailReduce = 0;
 constexpr int kDefaultChainPrefetch = 1;
+// gnorm_fwd_bwd / gnorm_ckpt_step: the (recompute) forward and the backward in one kernel,
+// which reads x, g and dy once for both.
+constexpr int kDefaultFuseFwdBwd = 1;
 constexpr int64_t kFusedReduceMaxFloats = 65536;
 
 struct RowGeometry {

@@ -19,6 +19,7 @@ __all__ = [
     "gnorm_fwd",
     "gnorm_bwd",
     "gnorm_ckpt_step",
+    "gnorm_fwd_bwd",
     "gnorm_ckpt_step_host",
     "gnorm_ckpt_step_host_bytes",
     "gnorm_bwd_noalloc",
@@ -93,7 +94,7 @@ def gnorm_selftest_wait_timeout(timeout_us: int = 20000) -> int:
 def gnorm_set_tuning(**knobs) -> None:
     """Process-wide experiment knobs (fields of gnorm_tuning; 0 = built-in).  No arguments
     restores every built-in choice.  Tri-state knobs (l2_prefetch, tail_reduce,
-    chain_prefetch, fwd_direct, bwd_direct): 1 on, 2 off, 0 built-in."""
+    chain_prefetch, fwd_direct, bwd_direct, fuse_fwd_bwd): 1 on, 2 off, 0 built-in."""
     t = GnormTuning()
     names = {f for f, _ in GnormTuning._fields_}
     for k, v in knobs.items():
@@ -298,6 +299,20 @@ def gnorm_ckpt_step(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=N
         st = lib.gnorm_ckpt_step_ex(ctypes.byref(fd), ctypes.byref(bd),
                                     _stream(stream, x.device))
     _check(st, "gnorm_ckpt_step")
+    return y, rstd, dx, dg, dw
+
+
+def gnorm_fwd_bwd(x, g, w, eps: float, dy, *, y=None, rstd=None, dx=None, dg=None, dw=None,
+                  dw_fp32: bool = False, deterministic: bool = True, workspace_buf=None,
+                  stream=None):
+    """Forward and backward of the same rows in one pass (the recompute forward of a
+    checkpointed layer and its backward): returns (y, rstd, dx, dg, dw)."""
+    fd, y, rstd = _fwd_desc(x, g, w, eps, y, rstd)
+    bd, dx, dg, dw = _bwd_desc(dy, x, g, w, rstd, dx, dg, dw, dw_fp32, deterministic,
+                               workspace_buf)
+    with torch.cuda.device(x.device):
+        st = lib.gnorm_fwd_bwd_ex(ctypes.byref(fd), ctypes.byref(bd), _stream(stream, x.device))
+    _check(st, "gnorm_fwd_bwd")
     return y, rstd, dx, dg, dw
 
 

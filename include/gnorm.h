@@ -196,12 +196,32 @@ GNORM_API int gnorm_ckpt_step_ex(const gnorm_fwd_desc* fwd, const gnorm_bwd_desc
  * all enqueued on `stream`.  Flashinfer PR #8701, section "How the tables were measured":
  * "ckptg" is the checkpointed step (2 x forward + backward), "stepg_f32" the same with an
  * FP32 dw.  y and rstd hold the second forward's outputs (bitwise equal to the first's);
- * the backward consumes that rstd.  Arguments as for gnorm_fwd and gnorm_bwd.
+ * the backward consumes that rstd.  The recompute forward and the backward run as
+ * gnorm_fwd_bwd (one kernel that reads x, g and dy once for both).  Arguments as for
+ * gnorm_fwd and gnorm_bwd.
  */
 GNORM_API int gnorm_ckpt_step(const void* x, const void* g, const void* w, float eps, const void* dy,
                     void* y, float* rstd, void* dx, void* dg, void* dw,
                     int dw_fp32, int deterministic, int64_t M, int64_t N,
                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Forward and backward of the same rows in one pass: the recompute forward of an
+ * activation-checkpointed layer followed by its backward (the last two calls of the pages'
+ * "ckptg", flashinfer PR #8701, section "How the tables were measured", which times them as
+ * separate calls; fusing them is this library's own).  Reads x, g, w and dy; writes the
+ * forward's outputs y and rstd and the backward's dx, dg and dw -- bitwise the values of
+ * gnorm_fwd followed by gnorm_bwd with the same arguments (dw too in deterministic mode) --
+ * while reading x and g once instead of twice and never reading rstd back: per row 12N + 4
+ * bytes of DRAM traffic instead of 16N + 8.  Where the backward's plan loads rows straight
+ * into registers (few rows per SM) it runs as those two kernels.  Arguments and workspace
+ * as for gnorm_ckpt_step (and gnorm_fwd_bwd_ex as for gnorm_ckpt_step_ex).
+ */
+GNORM_API int gnorm_fwd_bwd(const void* x, const void* g, const void* w, float eps, const void* dy,
+                            void* y, float* rstd, void* dx, void* dg, void* dw, int dw_fp32,
+                            int deterministic, int64_t M, int64_t N, void* workspace,
+                            size_t workspace_bytes, void* stream);
+GNORM_API int gnorm_fwd_bwd_ex(const gnorm_fwd_desc* fwd, const gnorm_bwd_desc* bwd, void* stream);
 
 /*
  * Checkpointed step on HOST buffers (no counterpart in the pages: an entry point for callers
@@ -329,6 +349,9 @@ typedef struct gnorm_tuning {
                             size, 2 always stage rows in shared memory (0: by rows per SM) */
   int bwd_direct;        /* backward of rows of N <= 256: 1 load straight into registers at any
                             size, 2 always stage rows in shared memory (0: by rows per SM) */
+  int fuse_fwd_bwd;      /* gnorm_fwd_bwd and the checkpointed step's recompute: 1 the forward
+                            and the backward in one kernel where the backward plan stages its
+                            rows, 2 always two kernels (0: built-in, fused) */
 } gnorm_tuning;
 
 GNORM_API void gnorm_set_tuning(const gnorm_tuning* tuning);

@@ -31,6 +31,8 @@ KNOB_SETS = [
     dict(fwd_direct=2),
     dict(bwd_direct=1),
     dict(bwd_direct=2),
+    dict(fuse_fwd_bwd=1, bwd_direct=2),
+    dict(fuse_fwd_bwd=2, bwd_direct=2),
 ]
 
 
