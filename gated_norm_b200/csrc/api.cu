@@ -231,9 +231,14 @@ int enqueue_fwd(const DeviceInfo& d, const gnorm_fwd_desc& f, cudaStream_t strea
 int enqueue_bwd(const DeviceInfo& d, const gnorm_bwd_desc& b, cudaStream_t stream,
                 bool prefetch = false, const gnorm_fwd_desc* fused = nullptr) {
   gnorm_plan plan;
-  int st = make_plan(1, b.M, b.N, b.deterministic, d.num_sms, d.smem_optin, &plan);
+  int st = make_plan(fused != nullptr ? 2 : 1, b.M, b.N, b.deterministic, d.num_sms,
+                     d.smem_optin, &plan);
   if (st != GNORM_OK) return st;
-  if (fused != nullptr && plan.direct_loads) return GNORM_ERR_UNSUPPORTED;
+  // The fused kernel is staged only, and its partial rows must fit the workspace sized for
+  // the backward's plan.
+  if (fused != nullptr &&
+      (plan.direct_loads || workspace_bytes_for(plan, b.N) > b.workspace_bytes))
+    return GNORM_ERR_UNSUPPORTED;
   uint8_t* wsb = static_cast<uint8_t*>(b.workspace);
   BwdArgs a;
   a.dy = static_cast<const uint16_t*>(b.dy);

@@ -53,7 +53,7 @@ RowGeometry geometry_for(int kind, int64_t N) {
   const int64_t n8 = N / 8;  // 16-byte chunks per row
   if (n8 <= 4) return {4, 1};
   if (n8 <= 8) return {8, 1};
-  if (n8 <= 16) return kind == 0 ? RowGeometry{8, 2} : RowGeometry{16, 1};
+  if (n8 <= 16) return kind == 1 ? RowGeometry{16, 1} : RowGeometry{8, 2};
   if (n8 <= 32) return {16, 2};
   if (n8 <= 64) return {32, 2};
   if (n8 <= 128) return {64, 2};
@@ -80,12 +80,16 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
               int smem_per_block, gnorm_plan* out) {
   if (out == nullptr) return GNORM_ERR_NULL;
   std::memset(out, 0, sizeof(*out));
-  if (kind != 0 && kind != 1) return GNORM_ERR_ARG;
+  if (kind != 0 && kind != 1 && kind != 2) return GNORM_ERR_ARG;
+  // kind 2, the forward fused into the backward (gnorm_fwd_bwd), is the backward kernel with
+  // its own row geometry for rows of N <= 128 (geometry_for); everything else as kind 1.
+  const int plan_kind = kind;
+  if (kind == 2) kind = 1;
   if (M < 0 || N < 8 || N > GNORM_N_MAX || (N % 8) != 0) return GNORM_ERR_SHAPE;
   if (num_sms <= 0) return GNORM_ERR_ARG;
   if (smem_per_block <= 0) smem_per_block = kB200SmemPerBlock;
 
-  RowGeometry geo = geometry_for(kind, N);
+  RowGeometry geo = geometry_for(plan_kind, N);
   RowGeometry dgeo = direct_geometry_for(N);
   if (g_knobs.threads_per_row > 0 && g_knobs.chunks_per_thread > 0) {
     geo = {g_knobs.threads_per_row, g_knobs.chunks_per_thread};
@@ -140,7 +144,7 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
                                                        ? g_knobs.ctas_per_sm
                                                        : kDirectBwdCtasPerSm);
     const int64_t blocks = ceil_div(M, rows_per_iter);
-    out->kind = 1;
+    out->kind = plan_kind;
     out->threads_per_row = geo.threads_per_row;
     out->chunks_per_thread = 1;
     out->consumer_threads = kDirectThreads;
@@ -212,7 +216,7 @@ int make_plan(int kind, int64_t M, int64_t N, int deterministic, int num_sms,
   const int64_t smem = kHeaderBytes + body;
   if (smem > smem_cta) return GNORM_ERR_UNSUPPORTED;
 
-  out->kind = kind;
+  out->kind = plan_kind;
   out->threads_per_row = geo.threads_per_row;
   out->chunks_per_thread = geo.chunks_per_thread;
   out->consumer_threads = nct;

@@ -294,7 +294,7 @@ GNORM_API const char* gnorm_status_string(int status);
  * (M / number of SMs) into tiers; this library's rule is its own, tuned for B200.
  */
 typedef struct gnorm_plan {
-  int kind;              /* 0 forward, 1 backward */
+  int kind;              /* 0 forward, 1 backward, 2 forward fused into the backward */
   int threads_per_row;   /* threads that share one row */
   int chunks_per_thread; /* 16-byte chunks (8 BF16 values) per thread and tensor */
   int consumer_threads;  /* computing threads per CTA (one extra warp issues the copies) */
@@ -313,7 +313,9 @@ typedef struct gnorm_plan {
 } gnorm_plan;
 
 /*
- * The dispatch rule as a pure host function: plan for `kind` (0 fwd, 1 bwd) on a device with
+ * The dispatch rule as a pure host function: plan for `kind` (0 fwd, 1 bwd, 2 the fused
+ * forward + backward of gnorm_fwd_bwd, which falls back to kinds 0 and 1 when its plan loads
+ * rows straight into registers) on a device with
  * `num_sms` SMs and `smem_per_block` bytes of opt-in shared memory per CTA (0 = 232448, the
  * B200 value).  Needs no GPU.  Returns GNORM_OK or an error status.
  */

@@ -212,8 +212,8 @@ def test_ctas_per_sm_never_exceeds_the_compiled_residency():
 def test_plan_errors():
     with pytest.raises(gn.GnormError):
         gn.gnorm_plan_query(0, 10, 12, True, 148)
-    with pytest.raises(gn.GnormError):
-        gn.gnorm_plan_query(2, 10, 128, True, 148)
+    with pytest.raises(gn.GnormError):  # kinds are 0 (forward), 1 (backward), 2 (fused)
+        gn.gnorm_plan_query(3, 10, 128, True, 148)
     with pytest.raises(gn.GnormError):
         gn.gnorm_plan_query(0, 10, 128, True, 0)
     with pytest.raises(gn.GnormError):  # shared memory too small for two stages of a row
@@ -374,3 +374,24 @@ def test_header_states_the_workspace_rule_after_a_timeout():
     text = open(os.path.join(ROOT, "include", "gnorm.h")).read()
     assert "zero the first GNORM_WORKSPACE_ALIGN bytes again" in text
     assert "every call that\n *   completes normally leaves them zero again" in text
+
+
+def test_fused_plan_is_the_backward_plan_with_its_own_narrow_geometry():
+    """Kind 2 (the forward fused into the backward) plans like the backward -- same CTAs,
+    blocks, stages, direct-load decision and partial rows, so the same workspace suffices --
+    except that rows of N <= 128 take 8 threads x 2 chunks (16 x 1 in the backward)."""
+    for sms in SM_COUNTS:
+        for M, N in ((368640, 128), (65536, 128), (4099, 64), (262144, 256), (16384, 4096),
+                     (1024, 128), (37, 8200)):
+            b = gn.gnorm_plan_query(1, M, N, True, sms)
+            f = gn.gnorm_plan_query(2, M, N, True, sms)
+            assert f["kind"] == 2
+            for k in ("rows_per_stage", "stages", "grid", "num_blocks", "direct_loads",
+                      "partials", "dynamic_schedule", "ctas_per_sm"):
+                assert f[k] == b[k], (M, N, k)
+            if 64 < N <= 128 and not f["direct_loads"]:
+                assert (f["threads_per_row"], f["chunks_per_thread"]) == (8, 2)
+                assert (b["threads_per_row"], b["chunks_per_thread"]) == (16, 1)
+            elif not f["direct_loads"]:
+                assert (f["threads_per_row"], f["chunks_per_thread"]) == \
+                    (b["threads_per_row"], b["chunks_per_thread"])
