@@ -94,7 +94,7 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectBwdCtasPerSm)
         const float2 sgm = sigmoid2(gp[i]);
         const float2 silu = mul2(gp[i], sgm);
         const float2 t = mul2(dyp[i], xhat);                 // dy xhat
-        ue[i] = mul2(mul2(dyp[i], wp[i]), silu);              // dy w s
+        ue[i] = mul2(dyp[i], mul2(wp[i], silu));              // dy (w s)
         xh[i] = xhat;
         if (valid[u]) dwacc[i] = fma2(t, silu, dwacc[i]);
         // sigmoid' = sigmoid (1 + g (1 - sigmoid))

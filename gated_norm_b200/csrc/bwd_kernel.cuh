@@ -192,6 +192,11 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
   constexpr int kNCT = consumer_threads_for(1, TPR, CPT);
   constexpr int kGroups = kNCT / TPR;
   constexpr bool kKeepXhat = kNCT <= 256 || CPT == 1;
+  // the fused forward's staged x, kept in registers from its row sum for pass 1.  Measured
+  // together with y and u sharing w s (against neither): faster with 16 or more threads per
+  // row (262144 x 256: 133.5 -> 129.9 us; 16384 x 4096: 145.6 -> 139.3 us), slower with 8
+  // (368640 x 128: 93.8 -> 97.9 us); not with four chunks per thread (register spills)
+  constexpr bool kKeepX = kFusedFwd && kKeepXhat && CPT <= 2 && TPR >= 16;
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);
   uint64_t* empty = full + kMaxStages;
@@ -373,6 +378,7 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
       const size_t roff = static_cast<size_t>(srow) * N * 2;
       const long long grow = r0 + row;
       float r;
+      float2 xs[CPT][4];  // the staged x as pairs (kKeepX)
       if constexpr (kFusedFwd) {
         // the forward's row sum: sum of squares of the staged x, one partial per chunk
         float sq[CPT];
@@ -380,11 +386,10 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
         for (int k = 0; k < CPT; ++k) {
           sq[k] = 0.f;
           if (cval[k]) {
-            float2 xp[4];
             bf16x8_to_pairs(
                 *reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(k * TPR + lr) * 16),
-                xp);
-            sq[k] = chunk_dot(xp, xp);
+                xs[k]);
+            sq[k] = chunk_dot(xs[k], xs[k]);
           }
         }
         const float ss = row_sum<TPR>(combine_chunks<CPT>(sq), red_slots, group, lr, slot);
@@ -408,16 +413,22 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
           const size_t off = roff + static_cast<size_t>(c) * 16;
           float2 dyp[4], xp[4], gp[4], dgp[4], yp[4];
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
-          bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
+          if constexpr (kKeepX) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) xp[i] = xs[k][i];
+          } else {
+            bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
+          }
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sg + off), gp);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 xhat = mul2(xp[i], r2);
             const float2 sgm = sigmoid2(gp[i]);
             const float2 silu = mul2(gp[i], sgm);
-            if constexpr (kFusedFwd) yp[i] = mul2(mul2(xhat, wp[k][i]), silu);  // the forward's y
+            const float2 ws = mul2(wp[k][i], silu);                 // w s
+            if constexpr (kFusedFwd) yp[i] = mul2(xhat, ws);        // the forward's y
             const float2 t = mul2(dyp[i], xhat);                    // dy xhat
-            const float2 ue = mul2(mul2(dyp[i], wp[k][i]), silu);    // dy w s
+            const float2 ue = mul2(dyp[i], ws);                     // dy (w s)
             u[k][i] = ue;
             xh[k][i] = xhat;
             if (valid) dwacc[k][i] = fma2(t, silu, dwacc[k][i]);

@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kDirectThreads, kDirectCtasPerSm)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const float2 silu = mul2(gp[i], sigmoid2(gp[i]));
-          yp[i] = mul2(mul2(mul2(xp[i], r2), wp[i]), silu);
+          yp[i] = mul2(mul2(xp[i], r2), mul2(wp[i], silu));
         }
         *(reinterpret_cast<uint4*>(a.y + row[u] * a.ldy) + lr) = pairs_to_bf16x8(yp);
       }

@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(consumer_threads_for(0, TPR, CPT) + 32, max_ct
       const long long grow = r0 + row;
       if (valid && lr == 0) a.rstd[grow] = r;
 
-      // pass 2: y = ((x r) w) (g sigmoid(g))
+      // pass 2: y = (x r) (w (g sigmoid(g)))
       const float2 r2 = splat2(r);
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(consumer_threads_for(0, TPR, CPT) + 32, max_ct
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             const float2 silu = mul2(gp[i], sigmoid2(gp[i]));
-            yp[i] = mul2(mul2(mul2(xp[i], r2), wp[k][i]), silu);
+            yp[i] = mul2(mul2(xp[i], r2), mul2(wp[k][i], silu));
           }
           if (valid)
             *reinterpret_cast<uint4*>(a.y + grow * a.ldy + c * 8) = pairs_to_bf16x8(yp);
