@@ -194,3 +194,22 @@ def test_workload_sampled(name):
             got = dev_to_f64(dw)
             rep = dw_fp32_check(got, dw_ref) if fp32 else bf16_check(got, dw_ref)
             assert rep["ok"], f"dw: {rep}"
+
+
+@pytest.mark.parametrize("name", ["long_368640x128", "wide_16384x4096", "mid_262144x256"])
+def test_workload_sampled_fused(name):
+    """The forward fused into the backward (gnorm_fwd_bwd, the checkpointed step's second
+    half, which the benchmark times at every large workload) at full size: sampled rows,
+    dw over all rows."""
+    case, wl = _workload_case(name)
+    rows = sample_rows(case.M, extra=case.host["outlier_rows"])
+    dw_ref = case.oracle_dw()
+    for det in wl.deterministic:
+        y, rstd, dx, dg, dw = gn.gnorm_fwd_bwd(case.x, case.g, case.w, case.eps, case.dy,
+                                               dw_fp32=True, deterministic=det)
+        torch.cuda.synchronize()
+        _check_fwd(case, y, rstd, rows)
+        _check_bwd(case, dx, dg, rows)
+        rep = dw_fp32_check(dev_to_f64(dw), dw_ref)
+        assert rep["ok"], f"dw: {rep}"
+    assert gn.gnorm_device_error(reset=True) == 0
