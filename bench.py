@@ -126,15 +126,24 @@ def measured_peaks():
 _DIGEST_EXCLUDED = ("host_step.cu", "noalloc.cu")
 
 
-def source_digest():
-    """Digest of the kernel sources and of the host code that plans and launches them."""
+def _code_only(text):
+    """C/C++/CUDA source without its comments and blank lines (the sources hold no string
+    literal with a comment marker), so that a comment edit keeps the digest."""
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.rstrip() for line in text.splitlines() if line.strip())
+
+
+def source_digest(csrc=None):
+    """Digest of the kernel sources and of the host code that plans and launches them
+    (their code, not their comments)."""
     h = hashlib.sha256()
-    csrc = os.path.join(ROOT, "gated_norm_b200", "csrc")
+    csrc = csrc or os.path.join(ROOT, "gated_norm_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name in _DIGEST_EXCLUDED:
             continue
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name), encoding="utf-8") as f:
+            h.update(name.encode() + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

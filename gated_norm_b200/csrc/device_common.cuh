@@ -105,8 +105,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, unsign
 }
 
 // 1-D bulk copy global -> shared through the TMA unit; completion is counted in bytes on
-// `bar`.  Both addresses must be 16-byte aligned and `bytes` a multiple of 16.  No
-// multicast: the source is always this GPU's memory and only this CTA receives it.
+// `bar`.  Both addresses must be 16-byte aligned and `bytes` a multiple of 16.  One
+// receiver: the source is always this GPU's memory and only this CTA receives it.
 __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_src,
                                               uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -117,7 +117,7 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
 }
 
 // Tiled 2-D TMA load of the box at (c0, c1) of `map` into shared memory (128-byte aligned),
-// completion counted in bytes on `bar`.  No multicast.
+// completion counted in bytes on `bar`; only this CTA receives the box.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int c0, int c1,
                                             uint64_t* bar) {
   asm volatile(
