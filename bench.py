@@ -4,17 +4,19 @@
                     [--workload NAME] [--nondeterministic] [--dw-bf16] [--flush]
 
 A step is one checkpointed training step over one batch of seeded synthetic rows:
-forward, forward again (recompute), backward with the dw reduction -- every stage of the
-path -- replayed from one CUDA graph ("ckptg").  The default workload is 262144 x 256 with
+forward, then the recompute forward and the backward (one kernel where the backward stages
+its rows) with the dw reduction -- every stage of the path -- replayed from one CUDA graph
+("ckptg").  The default workload is 262144 x 256 with
 an FP32 dw, deterministic (the checkpointed step with FP32 dw, "stepg_f32" in the pages'
 list of operations).  The timed region is K steps.  When the inputs are larger than L2
 (x and g alone exceed it at every large workload) the K replays run back to back between
 one pair of CUDA events; otherwise L2 is flushed before every replay, outside a pair of
-events around that replay.  After the timed region the forward ("fwdg") and the backward
-("bwdg") are timed the same way from their own graphs, for the per-operation times and the
-roofline of each; the three operations are also timed with a cold L2 before every replay
-(`us_per_call_cold_l2`), and `per_config` gives fwdg / bwdg / ckptg of the other large
-workloads.  `value` is the checkpointed step's algorithmic HBM bytes of the whole job / the
+events around that replay.  Before the timed region the forward ("fwdg"), the backward
+("bwdg") and the fused forward + backward are timed the same way from their own graphs, for
+the per-operation times and the roofline of each; after it the operations are also timed
+with a cold L2 before every replay (`us_per_call_cold_l2`), called eagerly through the
+Python binding without a graph (`us_per_call_eager`, the pages' "fwd" column), and
+`per_config` gives them for the other large workloads.  `value` is the checkpointed step's algorithmic HBM bytes of the whole job / the
 max-over-ranks time of the K steps (GB/s).
 
 Under torchrun (N > 1) every rank runs its own batch (weak scaling, no collective on the
@@ -334,6 +336,13 @@ def capture_graph(torch, dev, stream, fn, launches=1):
     return graph
 
 
+class _Eager:
+    """A callable with a graph's replay() interface, for Timer."""
+
+    def __init__(self, fn):
+        self.replay = fn
+
+
 class Timer:
     """CUDA-event timing of graph replays on `stream`.
 
@@ -548,6 +557,15 @@ def run_ours(args, wl):
     us_cold = {name: prob_t * 1e3 for name, prob_t in
                ((n, timer.cold(prob.graphs[n], cold_reps))
                 for n in ("fwd", "bwd", "fwd_bwd", "ckpt"))}
+    # the same operations called eagerly (no graph): each call goes through the binding and
+    # the C entry point, which plan and launch on the stream
+    eager_reps = max(10, min(K, OP_REPS))
+    us_eager = {}
+    for name, fn in (("fwd", prob.op_fwd), ("bwd", prob.op_bwd), ("fwd_bwd", prob.op_fwd_bwd),
+                     ("ckpt", prob.op_ckpt)):
+        call = _Eager(fn)
+        timer.run(call, 3)
+        us_eager[name] = timer.run(call, eager_reps)[0] / eager_reps * 1e3
     per_config = {}
     if args.per_config and world == 1:
         for name in PER_CONFIG_WORKLOADS:
@@ -695,6 +713,11 @@ def run_ours(args, wl):
         "cold_l2_note": (f"{cold_reps} replays each after a {flush.numel() >> 20} MiB L2 flush, "
                          "events around each replay, so each also counts its graph's launch "
                          "latency"),
+        "us_per_call_eager": us_eager,
+        "eager_note": (f"{eager_reps} calls of each operation through the Python binding "
+                       "without a graph, timed like the graph replays (back to back, or each "
+                       "after an L2 flush); each call's host path is in the time where it is "
+                       "longer than the kernels"),
         "roofline": roofline_of(dominant),
         "roofline_fwd": roofline_of("fwd"),
         "roofline_bwd": roofline_of("bwd"),
