@@ -191,7 +191,16 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
     gated_rmsnorm_bwd_kernel(const __grid_constant__ BwdArgs a) {
   constexpr int kNCT = consumer_threads_for(1, TPR, CPT);
   constexpr int kGroups = kNCT / TPR;
-  constexpr bool kKeepXhat = kNCT <= 256 || CPT == 1;
+  // xhat stays in registers from pass 1 to pass 2 with one or two chunks per thread; with
+  // four (rows wider than 4096) it is recomputed from the staged x, since keeping it spilled
+  // registers, and spills are slow next to ~200 KB of stages (8192 x 8192 backward 132 ->
+  // 113 us, fused forward + backward 226 -> 137 us without them)
+  constexpr bool kKeepXhat = (kNCT <= 256 && CPT <= 2) || CPT == 1;
+  // u = dy (w s) and the weights stay in registers too, except with 544 threads per CTA and
+  // four chunks per thread (rows wider than 8192), where the registers are capped at 96:
+  // each pass then reloads its chunk's weights and pass 2 recomputes u from the staged dy
+  // and g (the same operations, so the same bits)
+  constexpr bool kKeepU = kNCT <= 256 || CPT <= 2;
   // the fused forward's staged x, kept in registers from its row sum for pass 1.  Measured
   // together with y and u sharing w s (against neither): faster with 16 or more threads per
   // row (262144 x 256: 133.5 -> 129.9 us; 16384 x 4096: 145.6 -> 139.3 us), slower with 8
@@ -350,7 +359,8 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
       wp[k][i] = splat2(0.f);
       dwacc[k][i] = splat2(0.f);
     }
-    if (cval[k]) load_weight_pairs<kWFp32>(a.w, c, wp[k]);
+    if constexpr (kKeepU)  // else each pass reloads its chunk's weights (L1-resident)
+      if (cval[k]) load_weight_pairs<kWFp32>(a.w, c, wp[k]);
   }
 
   int s = 0;
@@ -402,8 +412,8 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
       const float2 r2 = splat2(r);
 
       // pass 1: recompute xhat and the gate; dg; row dot product; dw accumulators
-      float2 u[CPT][4];
-      float2 xh[CPT][4];  // xhat, kept for pass 2 where the registers allow it
+      float2 u[CPT][4];   // u, kept for pass 2 where the registers allow it (kKeepU)
+      float2 xh[CPT][4];  // xhat, likewise (kKeepXhat)
       float part[CPT];
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
@@ -411,7 +421,13 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
         if (cval[k]) {
           const int c = k * TPR + lr;
           const size_t off = roff + static_cast<size_t>(c) * 16;
-          float2 dyp[4], xp[4], gp[4], dgp[4], yp[4];
+          float2 dyp[4], xp[4], gp[4], dgp[4], yp[4], ul[4], xl[4], wk[4];
+          if constexpr (kKeepU) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wk[i] = wp[k][i];
+          } else {
+            load_weight_pairs<kWFp32>(a.w, c, wk);
+          }
           bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
           if constexpr (kKeepX) {
 #pragma unroll
@@ -425,18 +441,23 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
             const float2 xhat = mul2(xp[i], r2);
             const float2 sgm = sigmoid2(gp[i]);
             const float2 silu = mul2(gp[i], sgm);
-            const float2 ws = mul2(wp[k][i], silu);                 // w s
+            const float2 ws = mul2(wk[i], silu);                    // w s
             if constexpr (kFusedFwd) yp[i] = mul2(xhat, ws);        // the forward's y
             const float2 t = mul2(dyp[i], xhat);                    // dy xhat
             const float2 ue = mul2(dyp[i], ws);                     // dy (w s)
-            u[k][i] = ue;
-            xh[k][i] = xhat;
+            ul[i] = ue;
+            xl[i] = xhat;
             if (valid) dwacc[k][i] = fma2(t, silu, dwacc[k][i]);
             // sigmoid' = sigmoid (1 + g (1 - sigmoid))
             const float2 bracket = gate_grad_bracket(gp[i], sgm);
-            dgp[i] = mul2(mul2(mul2(t, wp[k][i]), sgm), bracket);
+            dgp[i] = mul2(mul2(mul2(t, wk[i]), sgm), bracket);
           }
-          part[k] = chunk_dot(u[k], xh[k]);  // this chunk's share of sum(u xhat)
+          part[k] = chunk_dot(ul, xl);  // this chunk's share of sum(u xhat)
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            if constexpr (kKeepU) u[k][i] = ul[i];
+            if constexpr (kKeepXhat) xh[k][i] = xl[i];
+          }
           if (valid) {
             *reinterpret_cast<uint4*>(a.dg + grow * a.lddg + c * 8) = pairs_to_bf16x8(dgp);
             if constexpr (kFusedFwd)
@@ -448,23 +469,35 @@ __global__ void __launch_bounds__(consumer_threads_for(1, TPR, CPT) + 32, max_ct
       slot ^= 1;
       const float2 nrc2 = splat2(-(r * (dot * a.inv_n)));
 
-      // pass 2: dx = r u - (r c) xhat.  xhat comes from pass 1's registers, except for the
-      // widest rows (544 threads per CTA cap the registers), which recompute it from the
-      // staged x -- the same product, so the same bits.
+      // pass 2: dx = r u - (r c) xhat.  xhat comes from pass 1's registers, except for rows
+      // of four chunks per thread (kKeepXhat), which recompute it from the staged x -- the
+      // same product, so the same bits.
 #pragma unroll
       for (int k = 0; k < CPT; ++k) {
         if (cval[k]) {
           const int c = k * TPR + lr;
           float2 dxp[4];
-          if constexpr (kKeepXhat) {
+          if constexpr (kKeepXhat && kKeepU) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) dxp[i] = fma2(nrc2, xh[k][i], mul2(r2, u[k][i]));
-          } else {
+          } else if constexpr (kKeepU) {
             float2 xp[4];
             bf16x8_to_pairs(
                 *reinterpret_cast<const uint4*>(sx + roff + static_cast<size_t>(c) * 16), xp);
 #pragma unroll
             for (int i = 0; i < 4; ++i) dxp[i] = fma2(nrc2, mul2(xp[i], r2), mul2(r2, u[k][i]));
+          } else {
+            const size_t off = roff + static_cast<size_t>(c) * 16;
+            float2 dyp[4], xp[4], gp[4], wk[4];
+            load_weight_pairs<kWFp32>(a.w, c, wk);
+            bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sdy + off), dyp);
+            bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sx + off), xp);
+            bf16x8_to_pairs(*reinterpret_cast<const uint4*>(sg + off), gp);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float2 ue = mul2(dyp[i], mul2(wk[i], mul2(gp[i], sigmoid2(gp[i]))));
+              dxp[i] = fma2(nrc2, mul2(xp[i], r2), mul2(r2, ue));
+            }
           }
           if (valid)
             *reinterpret_cast<uint4*>(a.dx + grow * a.lddx + c * 8) = pairs_to_bf16x8(dxp);
