@@ -21,9 +21,11 @@ if torch.cuda.is_available():
     import gated_norm_b200 as gn
 
 # every staged geometry of the backward: N <= 32, <= 64, <= 128, <= 256, <= 512, <= 1024,
-# <= 2048, <= 4096, <= 8192, <= 16384; ragged row counts; 700 x 4096 has many blocks per CTA
+# <= 2048, <= 4096 (also 2056), <= 8192 (6144, 8192: xhat recomputed in pass 2), <= 16384
+# (8200, 16384: u recomputed too); ragged row counts; 700 x 4096 has many blocks per CTA
 SHAPES = [(300, 32), (1000, 64), (4099, 128), (2500, 256), (777, 136), (600, 512), (333, 1024),
-          (129, 2056), (700, 4096), (37, 8200), (19, 16384), (70001, 128), (16385, 256)]
+          (97, 2048), (129, 2056), (700, 4096), (45, 6144), (23, 8192), (37, 8200), (19, 16384),
+          (70001, 128), (16385, 256)]
 
 
 def _bits(t):
